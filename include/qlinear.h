@@ -1,0 +1,164 @@
+/*
+ * qlinear.h -- C ABI of the B200 (sm_100a) dynamically quantized linear layer.
+ *
+ * One linear layer of a diffusion-transformer denoising step, in three parts:
+ *   1. activation quantization, per call (qlinear_quantize_act):
+ *        FP8  : per-token E4M3 codes with an fp32 scale per row (amax/448);
+ *        NVFP4: E2M1 codes in 16-element K blocks, an E4M3 scale per block and
+ *               an fp32 global scale for the tensor (amax/2688);
+ *   2. a block-scaled tensor-core GEMM of those codes against weights that
+ *      were quantized once by qlinear_create (same formats; FP8 weights carry
+ *      one fp32 scale per output channel);
+ *   3. a fused epilogue: dequantization scale, bias, then GELU-tanh, SwiGLU or
+ *      an adaLN-gated residual add, and a bf16 store (qlinear_forward).
+ *
+ * Sources: "Cuantizacion Dinamica FP8" in wavespeed.ai's "Solucion de
+ * WaveSpeed para Acelerar la Generacion de Imagenes FLUX.1-dev" (weights and
+ * activations lowered to FP8 with run-time scales, matmul on the 8-bit tensor
+ * cores); algoritmulzilei.ro, "Accelerarea generarii de imagini cu FLUX 3 Image
+ * Klein pe GPU-urile Blackwell" (NVFP4 DiT; GEMMs with fused epilogues such as
+ * SwiGLU); bytechap.com, "Optimizacion de la inferencia de FLUX 3 Image Klein",
+ * section "Como funciona" (NVFP4 lowers both weights and activations).  The
+ * pages give no API; this one follows the three-call structure of the path.
+ *
+ * Conventions for every call:
+ *   - All device memory is owned by the caller.  The library never allocates
+ *     device memory and never synchronizes the host in the launch calls
+ *     (qlinear_quantize_act, qlinear_forward).
+ *   - Device pointers must be 16-byte aligned (QL_ERR_ALIGNMENT otherwise).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   - Argument errors are returned before anything is launched.  Launch
+ *     failures return QL_ERR_CUDA.  A device-side bounded wait that expired
+ *     (the GEMM's pipeline watchdog, about one second) is reported as
+ *     QL_ERR_TIMEOUT by the next qlinear_check on the handle.
+ *   - bf16 tensors are row-major with unit inner stride.
+ *   - A handle may be used from one host thread at a time.
+ */
+#ifndef QLINEAR_H
+#define QLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QL_API __attribute__((visibility("default")))
+#else
+#define QL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct qlinear_s* qlinear_t;
+
+typedef enum {
+  QL_OK = 0,
+  QL_ERR_INVALID_ARG = 1, /* null pointer, bad shape/enum, size too small      */
+  QL_ERR_ALIGNMENT = 2,   /* pointer or leading dimension not 16-byte aligned  */
+  QL_ERR_UNSUPPORTED = 3, /* valid but not supported (e.g. no sm_100 device)   */
+  QL_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed                 */
+  QL_ERR_TIMEOUT = 5      /* a device-side bounded wait expired                */
+} ql_status;
+
+typedef enum { QL_FP8_E4M3 = 0, QL_NVFP4 = 1 } ql_format;
+
+typedef enum {
+  QL_EPI_BIAS = 0,                 /* out = y + b                                  */
+  QL_EPI_BIAS_GELU = 1,            /* out = gelu_tanh(y + b)                       */
+  QL_EPI_SWIGLU = 2,               /* out[:,j] = silu(y[:,j]+b[j]) * (y[:,Nout+j]+b[Nout+j]),
+                                      N = 2*Nout, weight rows [0,Nout) = gate,
+                                      [Nout,N) = up                                */
+  QL_EPI_BIAS_GATED_RESIDUAL = 3,  /* out = residual + gate[n] * (y + b)  (adaLN)  */
+  QL_EPI_SPLIT_BIAS_GELU = 4       /* n < split_col: y + b ; else gelu_tanh(y + b) */
+} ql_epilogue;
+
+/* Layer description.  y = dequant(codes_x) @ dequant(codes_w)^T, shape [M, N]. */
+typedef struct {
+  int32_t fmt;       /* ql_format                                                */
+  int32_t epi;       /* ql_epilogue                                              */
+  int64_t N;         /* output features of the GEMM (SwiGLU: 2*Nout)             */
+  int64_t K;         /* input features                                           */
+  int64_t split_col; /* QL_EPI_SPLIT_BIAS_GELU only: first GELU column           */
+  int32_t variant;   /* 0 = default kernel configuration                         */
+  int32_t flags;     /* must be 0                                                */
+} ql_desc;
+
+/* Shape rules (QL_ERR_INVALID_ARG otherwise):
+ *   FP8  : K % 16 == 0, N % 32 == 0;  NVFP4: K % 32 == 0, N % 256 == 0;
+ *   SwiGLU: N % 256 == 0;  1 <= K <= 2^24, 1 <= N <= 2^24, 0 <= M <= 2^31-1;
+ *   split_col % 32 == 0 for the split epilogue.
+ */
+
+/* Bytes of device workspace the handle needs (weights codes + scales + bias +
+ * a small control block).  Host only, no CUDA call. */
+QL_API ql_status qlinear_weight_bytes(const ql_desc* desc, size_t* bytes);
+
+/* Quantize W once and lay it out for the GEMM.
+ *   w_bf16    : device, [N, K] bf16 master weights (read only during the call's
+ *               kernels; may be freed once the stream has passed them).
+ *   bias_bf16 : device, [N] bf16, or NULL for zero bias.  Copied into weight_ws.
+ *   weight_ws : device, >= qlinear_weight_bytes(desc), 256-byte aligned; must
+ *               stay alive and untouched until qlinear_destroy.
+ *   stream    : the kernels are enqueued here; the handle may be used on any
+ *               stream ordered after this one.
+ *   out       : receives the handle (host object owned by the library).
+ * FP8 weights: per output channel n, s_w[n] = amax/448, codes E4M3(w*448/amax).
+ * NVFP4 weights: global scale over all of W, 16-element block scales. */
+QL_API ql_status qlinear_create(const ql_desc* desc, const void* w_bf16, const void* bias_bf16,
+                         void* weight_ws, size_t ws_bytes, void* stream, qlinear_t* out);
+
+/* Sizes of the activation code and scale buffers for M tokens.
+ *   FP8  : codes [M, K] bytes; scales fp32 [M] (rounded up to 16 bytes).
+ *   NVFP4: codes [M, K/2] bytes (two codes per byte, low nibble first);
+ *          scales = block scales in the GEMM's tiled layout
+ *          (ceil(M/128) x ceil(K/256)*4 chunks of 512 bytes) followed by a
+ *          16-byte tail holding the fp32 global scale and the amax word. */
+QL_API ql_status qlinear_act_bytes(qlinear_t h, int64_t M, size_t* code_bytes, size_t* scale_bytes);
+
+/* Number of output columns of qlinear_forward (N, or N/2 for SwiGLU). */
+QL_API ql_status qlinear_out_features(qlinear_t h, int64_t* nout);
+
+/* Dynamic activation quantization (no host sync, no allocation).
+ *   x_bf16 : device [M, K] bf16;  codes, scales: device, sized by
+ *   qlinear_act_bytes.  FP8: one fused pass (row amax, scale, cast).
+ *   NVFP4: a tensor-amax pass, then the block quantize that also writes the
+ *   global scale into the scales tail. */
+QL_API ql_status qlinear_quantize_act(qlinear_t h, const void* x_bf16, int64_t M, void* codes,
+                               void* scales, void* stream);
+
+/* GEMM + fused epilogue (no host sync, no allocation).
+ *   codes, scales : as written by qlinear_quantize_act for the same M.
+ *   residual      : device [M, Nout] bf16 for QL_EPI_BIAS_GATED_RESIDUAL, else NULL.
+ *   gate          : device [Nout] bf16 for QL_EPI_BIAS_GATED_RESIDUAL, else NULL.
+ *   out_bf16      : device [M, Nout] bf16 (Nout % 8 == 0). */
+QL_API ql_status qlinear_forward(qlinear_t h, const void* codes, const void* scales, int64_t M,
+                          const void* residual, const void* gate, void* out_bf16,
+                          void* stream);
+
+/* Copy the quantized weights to host memory in logical order (synchronizes).
+ *   FP8  : codes_host [N, K] bytes, scales_host fp32 [N], global_scale ignored.
+ *   NVFP4: codes_host [N, K/2] bytes, scales_host [N, K/16] E4M3 block-scale
+ *          codes, *global_scale = fp32 global scale. */
+QL_API ql_status qlinear_export_weights(qlinear_t h, void* codes_host, void* scales_host,
+                                 float* global_scale, void* stream);
+
+/* Synchronize `stream` and report a device-side error recorded for this
+ * handle (QL_ERR_TIMEOUT) or a pending CUDA error (QL_ERR_CUDA).  Clears the
+ * recorded error. */
+QL_API ql_status qlinear_check(qlinear_t h, void* stream);
+
+/* Release the host handle (the caller frees weight_ws afterwards). */
+QL_API ql_status qlinear_destroy(qlinear_t h);
+
+/* Static description of a status code. */
+QL_API const char* qlinear_status_string(ql_status s);
+
+/* ABI version of this header (incremented on incompatible changes). */
+QL_API int32_t qlinear_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLINEAR_H */

@@ -1,0 +1,99 @@
+"""B200 (sm_100a) dynamically quantized linear layer: FP8-E4M3 / NVFP4.
+
+The compute path is the C ABI in ``include/qlinear.h`` (``libqlinear_b200.so``,
+hand-written CUDA for sm_100a).  This package is a thin binding: ``_abi``
+marshals arguments to the C calls, and :class:`QLinear` owns the device
+buffers (allocated with PyTorch) and passes their pointers through.  No step
+of the path runs in Python or PyTorch.
+"""
+import numpy as np
+
+from . import _abi
+from ._abi import (EPILOGUES, FORMATS, QLinearError, make_desc, qlinear_abi_version,  # noqa: F401
+                   qlinear_act_bytes, qlinear_check, qlinear_create, qlinear_destroy,
+                   qlinear_export_weights, qlinear_forward, qlinear_out_features,
+                   qlinear_quantize_act, qlinear_weight_bytes, status_string)
+
+__all__ = ["QLinear", "make_desc", "QLinearError"]
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+class QLinear:
+    """One quantized linear layer: weights quantized once, activations per call.
+
+    ``w`` is a bf16 CUDA tensor [N, K]; ``bias`` bf16 [N] or None.  The
+    workspace is a uint8 CUDA tensor owned by this object.
+    """
+
+    def __init__(self, fmt, epi, w, bias=None, split_col=0, stream=None):
+        import torch
+        assert w.is_cuda and w.dtype == torch.bfloat16 and w.is_contiguous()
+        N, K = w.shape
+        self.fmt, self.epi, self.N, self.K = fmt, epi, int(N), int(K)
+        self.desc = make_desc(fmt, epi, N, K, split_col)
+        nbytes = qlinear_weight_bytes(self.desc)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=w.device)
+        self.h = qlinear_create(self.desc, w.data_ptr(), _ptr(bias), self.ws.data_ptr(), nbytes,
+                                _stream_ptr(stream))
+        self.Nout = qlinear_out_features(self.h)
+
+    def act_buffers(self, M, device="cuda"):
+        import torch
+        cb, sb = qlinear_act_bytes(self.h, M)
+        return (torch.empty(max(cb, 16), dtype=torch.uint8, device=device),
+                torch.empty(max(sb, 16), dtype=torch.uint8, device=device))
+
+    def quantize(self, x, codes, scales, stream=None):
+        M = x.shape[0]
+        qlinear_quantize_act(self.h, x.data_ptr(), M, codes.data_ptr(), scales.data_ptr(),
+                             _stream_ptr(stream))
+
+    def forward_codes(self, codes, scales, M, out, residual=None, gate=None, stream=None):
+        qlinear_forward(self.h, codes.data_ptr(), scales.data_ptr(), M, _ptr(residual), _ptr(gate),
+                        out.data_ptr(), _stream_ptr(stream))
+
+    def __call__(self, x, residual=None, gate=None, out=None, bufs=None, stream=None):
+        import torch
+        M = x.shape[0]
+        codes, scales = bufs if bufs is not None else self.act_buffers(M, x.device)
+        if out is None:
+            out = torch.empty((M, self.Nout), dtype=torch.bfloat16, device=x.device)
+        self.quantize(x, codes, scales, stream)
+        self.forward_codes(codes, scales, M, out, residual, gate, stream)
+        return out
+
+    def export_weights(self):
+        """Quantized weights in logical order: (codes, scales, global_scale)."""
+        if self.fmt == "fp8":
+            codes = np.empty((self.N, self.K), np.uint8)
+            scales = np.empty(self.N, np.float32)
+        else:
+            codes = np.empty((self.N, self.K // 2), np.uint8)
+            scales = np.empty((self.N, self.K // 16), np.uint8)
+        g = qlinear_export_weights(self.h, codes.ctypes.data, scales.ctypes.data,
+                                   _stream_ptr(None))
+        return codes, scales, np.float32(g)
+
+    def check(self, stream=None):
+        return qlinear_check(self.h, _stream_ptr(stream))
+
+    def close(self):
+        if getattr(self, "h", None):
+            qlinear_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,414 @@
+// qlinear_api.cu -- the C ABI (include/qlinear.h): argument checks, weight
+// workspace layout, tensor-map encoding and kernel launches.  No device
+// allocation and no host synchronization in the launch calls.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "../../include/qlinear.h"
+#include "internal.h"
+
+using namespace qlb;
+
+struct qlinear_s {
+  ql_desc d;
+  int64_t N, K, Nout;
+  int device, num_sms;
+  uint8_t* ws;
+  size_t ws_bytes;
+  // workspace views
+  uint32_t* err;
+  uint8_t* wcodes;
+  float* wscale;     // FP8 per-channel scales [N]
+  uint8_t* wsf;      // NVFP4 scale-factor atoms
+  float* wG;         // NVFP4 global scale (device scalar)
+  uint32_t* wamax;   // NVFP4 amax word used while quantizing W
+  __nv_bfloat16* bias;
+  RowMap map;
+  CUtensorMap tmB;
+};
+
+namespace {
+
+constexpr int32_t kAbiVersion = 1;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+struct WsLayout {
+  size_t err, codes, scales, bias, total;
+};
+
+// Weight workspace: [control 256 B][codes][scales (+16 B tail for NVFP4)][bias]
+WsLayout ws_layout(const ql_desc& d) {
+  WsLayout L;
+  L.err = 0;
+  size_t off = 1024;
+  L.codes = off;
+  const size_t code_bytes = d.fmt == QL_NVFP4 ? static_cast<size_t>(d.N) * d.K / 2
+                                              : static_cast<size_t>(d.N) * d.K;
+  off = align_up(off + code_bytes, 1024);
+  L.scales = off;
+  const size_t sc_bytes = d.fmt == QL_NVFP4 ? static_cast<size_t>(sf_bytes(d.N, d.K)) + 16
+                                            : static_cast<size_t>(d.N) * 4;
+  off = align_up(off + sc_bytes, 1024);
+  L.bias = off;
+  off = align_up(off + static_cast<size_t>(d.N) * 2, 1024);
+  L.total = off;
+  return L;
+}
+
+ql_status check_desc(const ql_desc* d) {
+  if (!d) return QL_ERR_INVALID_ARG;
+  if (d->fmt != QL_FP8_E4M3 && d->fmt != QL_NVFP4) return QL_ERR_INVALID_ARG;
+  if (d->epi < QL_EPI_BIAS || d->epi > QL_EPI_SPLIT_BIAS_GELU) return QL_ERR_INVALID_ARG;
+  if (d->flags != 0 || d->variant != 0) return QL_ERR_INVALID_ARG;
+  if (d->N < 1 || d->K < 1 || d->N > (1 << 24) || d->K > (1 << 24)) return QL_ERR_INVALID_ARG;
+  if (d->N % 32 != 0) return QL_ERR_INVALID_ARG;
+  if (d->fmt == QL_FP8_E4M3 && d->K % 16 != 0) return QL_ERR_INVALID_ARG;
+  if (d->fmt == QL_NVFP4 && (d->K % 32 != 0 || d->N % 256 != 0)) return QL_ERR_INVALID_ARG;
+  if (d->epi == QL_EPI_SWIGLU && d->N % 256 != 0) return QL_ERR_INVALID_ARG;
+  if (d->epi == QL_EPI_SPLIT_BIAS_GELU &&
+      (d->split_col < 0 || d->split_col > d->N || d->split_col % 32 != 0))
+    return QL_ERR_INVALID_ARG;
+  return QL_OK;
+}
+
+struct DevInfo {
+  int device = -1;
+  int num_sms = 0;
+  int major = 0, minor = 0;
+};
+
+ql_status current_device(DevInfo* out) {
+  static std::mutex mu;
+  static std::vector<DevInfo> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto& c : cache)
+    if (c.device == dev) {
+      *out = c;
+      return QL_OK;
+    }
+  DevInfo di;
+  di.device = dev;
+  if (cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&di.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&di.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  cache.push_back(di);
+  *out = di;
+  return QL_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D tensor map over a row-major [outer, inner] array.
+bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+               uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+ql_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return QL_OK;
+  return QL_ERR_CUDA;
+}
+
+size_t act_code_bytes(const qlinear_s* h, int64_t M) {
+  return h->d.fmt == QL_NVFP4 ? static_cast<size_t>(M) * h->K / 2 : static_cast<size_t>(M) * h->K;
+}
+
+size_t act_scale_bytes(const qlinear_s* h, int64_t M) {
+  if (h->d.fmt == QL_NVFP4) return static_cast<size_t>(sf_bytes(M, h->K)) + 16;
+  return align_up(static_cast<size_t>(M) * 4, 16);
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t qlinear_abi_version(void) { return kAbiVersion; }
+
+const char* qlinear_status_string(ql_status s) {
+  switch (s) {
+    case QL_OK: return "ok";
+    case QL_ERR_INVALID_ARG: return "invalid argument";
+    case QL_ERR_ALIGNMENT: return "pointer or leading dimension not 16-byte aligned";
+    case QL_ERR_UNSUPPORTED: return "unsupported device or configuration";
+    case QL_ERR_CUDA: return "CUDA error";
+    case QL_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+ql_status qlinear_weight_bytes(const ql_desc* desc, size_t* bytes) {
+  if (!bytes) return QL_ERR_INVALID_ARG;
+  ql_status s = check_desc(desc);
+  if (s != QL_OK) return s;
+  *bytes = ws_layout(*desc).total;
+  return QL_OK;
+}
+
+ql_status qlinear_create(const ql_desc* desc, const void* w_bf16, const void* bias_bf16,
+                         void* weight_ws, size_t ws_bytes, void* stream, qlinear_t* out) {
+  if (!out) return QL_ERR_INVALID_ARG;
+  *out = nullptr;
+  ql_status s = check_desc(desc);
+  if (s != QL_OK) return s;
+  if (!w_bf16 || !weight_ws) return QL_ERR_INVALID_ARG;
+  if (!aligned16(w_bf16) || (bias_bf16 && !aligned16(bias_bf16)) ||
+      (reinterpret_cast<uintptr_t>(weight_ws) & 255) != 0)
+    return QL_ERR_ALIGNMENT;
+  const WsLayout L = ws_layout(*desc);
+  if (ws_bytes < L.total) return QL_ERR_INVALID_ARG;
+  DevInfo di;
+  if ((s = current_device(&di)) != QL_OK) return s;
+  if (di.major != 10) return QL_ERR_UNSUPPORTED;
+
+  qlinear_s* h = new (std::nothrow) qlinear_s();
+  if (!h) return QL_ERR_INVALID_ARG;
+  h->d = *desc;
+  h->N = desc->N;
+  h->K = desc->K;
+  h->Nout = desc->epi == QL_EPI_SWIGLU ? desc->N / 2 : desc->N;
+  h->device = di.device;
+  h->num_sms = di.num_sms;
+  h->ws = static_cast<uint8_t*>(weight_ws);
+  h->ws_bytes = ws_bytes;
+  h->err = reinterpret_cast<uint32_t*>(h->ws + L.err);
+  h->wcodes = h->ws + L.codes;
+  h->bias = reinterpret_cast<__nv_bfloat16*>(h->ws + L.bias);
+  h->map.nout = h->Nout;
+  h->map.mode = desc->epi == QL_EPI_SWIGLU ? 1 : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  cudaError_t e = cudaMemsetAsync(h->ws, 0, 1024, st);
+  if (e == cudaSuccess && desc->fmt == QL_FP8_E4M3) {
+    h->wscale = reinterpret_cast<float*>(h->ws + L.scales);
+    e = launch_quant_fp8_rows(w_bf16, h->N, h->K, h->K, h->wcodes, h->wscale, h->map, h->num_sms,
+                              st);
+  } else if (e == cudaSuccess) {
+    h->wsf = h->ws + L.scales;
+    h->wG = reinterpret_cast<float*>(h->wsf + sf_bytes(h->N, h->K));
+    h->wamax = reinterpret_cast<uint32_t*>(h->wG + 1);
+    e = cudaMemsetAsync(h->wamax, 0, 4, st);
+    if (e == cudaSuccess) e = launch_tensor_amax(w_bf16, h->N * h->K, h->wamax, h->num_sms, st);
+    if (e == cudaSuccess)
+      e = launch_quant_nvfp4(w_bf16, h->N, h->K, h->K, h->wcodes, h->wsf, h->wamax, h->wG, h->map,
+                             st);
+  }
+  if (e == cudaSuccess) e = launch_permute_bias(bias_bf16, h->bias, h->N, h->map, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return QL_ERR_CUDA;
+  }
+  const uint64_t kbytes = desc->fmt == QL_NVFP4 ? h->K / 2 : h->K;
+  if (!make_tmap(&h->tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, 128, 256,
+                 CU_TENSOR_MAP_SWIZZLE_128B)) {
+    delete h;
+    return QL_ERR_CUDA;
+  }
+  *out = h;
+  return QL_OK;
+}
+
+ql_status qlinear_act_bytes(qlinear_t h, int64_t M, size_t* code_bytes, size_t* scale_bytes) {
+  if (!h || M < 0 || M > 0x7FFFFFFF || !code_bytes || !scale_bytes) return QL_ERR_INVALID_ARG;
+  *code_bytes = act_code_bytes(h, M);
+  *scale_bytes = act_scale_bytes(h, M);
+  return QL_OK;
+}
+
+ql_status qlinear_out_features(qlinear_t h, int64_t* nout) {
+  if (!h || !nout) return QL_ERR_INVALID_ARG;
+  *nout = h->Nout;
+  return QL_OK;
+}
+
+ql_status qlinear_quantize_act(qlinear_t h, const void* x_bf16, int64_t M, void* codes,
+                               void* scales, void* stream) {
+  if (!h || M < 0 || M > 0x7FFFFFFF) return QL_ERR_INVALID_ARG;
+  if (M == 0) return QL_OK;
+  if (!x_bf16 || !codes || !scales) return QL_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scales)) return QL_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (h->d.fmt == QL_FP8_E4M3) {
+    e = launch_quant_fp8_rows(x_bf16, M, h->K, h->K, static_cast<uint8_t*>(codes),
+                              static_cast<float*>(scales), RowMap{0, 0}, h->num_sms, st);
+  } else {
+    uint8_t* sf = static_cast<uint8_t*>(scales);
+    float* g = reinterpret_cast<float*>(sf + sf_bytes(M, h->K));
+    uint32_t* amax = reinterpret_cast<uint32_t*>(g + 1);
+    e = cudaMemsetAsync(amax, 0, 4, st);
+    if (e == cudaSuccess) e = launch_tensor_amax(x_bf16, M * h->K, amax, h->num_sms, st);
+    if (e == cudaSuccess)
+      e = launch_quant_nvfp4(x_bf16, M, h->K, h->K, static_cast<uint8_t*>(codes), sf, amax, g,
+                             RowMap{0, 0}, st);
+  }
+  if (e != cudaSuccess) cudaGetLastError();
+  return from_cuda(e);
+}
+
+ql_status qlinear_forward(qlinear_t h, const void* codes, const void* scales, int64_t M,
+                          const void* residual, const void* gate, void* out_bf16, void* stream) {
+  if (!h || M < 0 || M > 0x7FFFFFFF) return QL_ERR_INVALID_ARG;
+  if (M == 0) return QL_OK;
+  if (!codes || !scales || !out_bf16) return QL_ERR_INVALID_ARG;
+  const bool gated = h->d.epi == QL_EPI_BIAS_GATED_RESIDUAL;
+  if (gated && (!residual || !gate)) return QL_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(out_bf16)) return QL_ERR_ALIGNMENT;
+  if (gated && (!aligned16(residual) || !aligned16(gate))) return QL_ERR_ALIGNMENT;
+  if (h->Nout % 8 != 0) return QL_ERR_ALIGNMENT;
+
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  const bool nv = h->d.fmt == QL_NVFP4;
+  const uint64_t kbytes = nv ? h->K / 2 : h->K;
+  if (!make_tmap(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, kbytes, M, kbytes, 128, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&p.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out_bf16, h->Nout, M, h->Nout * 2, 32,
+                 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return QL_ERR_CUDA;
+  p.tmB = h->tmB;
+  if (nv) {
+    p.sfa = static_cast<const uint8_t*>(scales);
+    p.ga = reinterpret_cast<const float*>(p.sfa + sf_bytes(M, h->K));
+    p.sfb = h->wsf;
+    p.gw = h->wG;
+  } else {
+    p.sa = static_cast<const float*>(scales);
+    p.sw = h->wscale;
+  }
+  p.bias = h->bias;
+  p.residual = static_cast<const __nv_bfloat16*>(residual);
+  p.gate = static_cast<const __nv_bfloat16*>(gate);
+  p.err = h->err;
+  p.M = static_cast<int32_t>(M);
+  p.N = static_cast<int32_t>(h->N);
+  p.Nout = static_cast<int32_t>(h->Nout);
+  p.split_col = static_cast<int32_t>(h->d.split_col);
+  p.k_blocks = static_cast<int32_t>((kbytes + 127) / 128);
+  p.tiles_m = static_cast<int32_t>((M + 127) / 128);
+  p.tiles_n = static_cast<int32_t>((h->N + 255) / 256);
+  p.group_m = 8;
+  p.sf_kchunks_a = static_cast<int32_t>(sf_kchunks(h->K));
+  p.sf_kchunks_b = static_cast<int32_t>(sf_kchunks(h->K));
+  p.fault_mode = 0;
+  cudaError_t e = launch_gemm(h->d.fmt, h->d.epi, p, h->num_sms, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
+}
+
+ql_status qlinear_export_weights(qlinear_t h, void* codes_host, void* scales_host,
+                                 float* global_scale, void* stream) {
+  if (!h || !codes_host || !scales_host) return QL_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  const bool nv = h->d.fmt == QL_NVFP4;
+  const size_t row_bytes = nv ? h->K / 2 : h->K;
+  std::vector<uint8_t> codes(static_cast<size_t>(h->N) * row_bytes);
+  if (cudaMemcpy(codes.data(), h->wcodes, codes.size(), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  uint8_t* ch = static_cast<uint8_t*>(codes_host);
+  for (int64_t p = 0; p < h->N; ++p)
+    std::memcpy(ch + h->map(p) * row_bytes, codes.data() + p * row_bytes, row_bytes);
+  if (!nv) {
+    std::vector<float> sc(h->N);
+    if (cudaMemcpy(sc.data(), h->wscale, h->N * 4, cudaMemcpyDeviceToHost) != cudaSuccess) {
+      cudaGetLastError();
+      return QL_ERR_CUDA;
+    }
+    float* sh = static_cast<float*>(scales_host);
+    for (int64_t p = 0; p < h->N; ++p) sh[h->map(p)] = sc[p];
+  } else {
+    std::vector<uint8_t> sf(sf_bytes(h->N, h->K));
+    float g = 0.f;
+    if (cudaMemcpy(sf.data(), h->wsf, sf.size(), cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemcpy(&g, h->wG, 4, cudaMemcpyDeviceToHost) != cudaSuccess) {
+      cudaGetLastError();
+      return QL_ERR_CUDA;
+    }
+    const int64_t nb = h->K / 16, kch = sf_kchunks(h->K);
+    uint8_t* sh = static_cast<uint8_t*>(scales_host);
+    for (int64_t p = 0; p < h->N; ++p)
+      for (int64_t b = 0; b < nb; ++b) sh[h->map(p) * nb + b] = sf[sf_offset(p, b, kch)];
+    if (global_scale) *global_scale = g;
+  }
+  return QL_OK;
+}
+
+ql_status qlinear_check(qlinear_t h, void* stream) {
+  if (!h) return QL_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  uint32_t err = 0;
+  if (cudaMemcpy(&err, h->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  if (err != 0) {
+    uint32_t zero = 0;
+    cudaMemcpy(h->err, &zero, 4, cudaMemcpyHostToDevice);
+    return QL_ERR_TIMEOUT;
+  }
+  return QL_OK;
+}
+
+ql_status qlinear_destroy(qlinear_t h) {
+  if (!h) return QL_ERR_INVALID_ARG;
+  delete h;
+  return QL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,251 @@
+// quant.cu -- dynamic activation / weight quantization kernels (HBM bound).
+//
+//  * quant_fp8_rows: per-token (per-row) FP8-E4M3.  One pass over the row:
+//    128-bit loads kept in registers, warp-shuffle (redux) amax, scale
+//    s = amax/448, inverse 448/amax, codes E4M3(x * inv) written as 64-bit
+//    stores.  "Cuantizacion Dinamica FP8", wavespeed.ai "Solucion de WaveSpeed
+//    para Acelerar la Generacion de Imagenes FLUX.1-dev".
+//  * tensor_amax + quant_nvfp4: NVFP4 two-level scaling (algoritmulzilei.ro,
+//    "Accelerarea generarii de imagini cu FLUX 3 Image Klein"; bytechap.com
+//    "Como funciona"): global scale G = A/2688 over the tensor, E4M3 block
+//    scale per 16 K-elements, packed E2M1 codes; block scales are written
+//    straight into the GEMM's scale-factor atom layout.
+//
+// Every float step is an explicitly rounded IEEE operation (__fmul_rn /
+// __fdiv_rn) so no FMA contraction changes a code.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace qlb {
+
+namespace {
+
+__device__ __forceinline__ float absmax8(const uint4& v) {
+  // |bf16| max over 8 values, done on the bit patterns' float images
+  float m = fmaxf(fabsf(bf16lo(v.x)), fabsf(bf16hi(v.x)));
+  m = fmaxf(m, fmaxf(fabsf(bf16lo(v.y)), fabsf(bf16hi(v.y))));
+  m = fmaxf(m, fmaxf(fabsf(bf16lo(v.z)), fabsf(bf16hi(v.z))));
+  m = fmaxf(m, fmaxf(fabsf(bf16lo(v.w)), fabsf(bf16hi(v.w))));
+  return m;
+}
+
+__device__ __forceinline__ uint32_t e4m3_pair(uint32_t w, float inv) {
+  // bf16x2 word -> 2 E4M3 codes (element 0 in the low byte)
+  return cvt_e4m3x2(__fmul_rn(bf16hi(w), inv), __fmul_rn(bf16lo(w), inv));
+}
+
+__device__ __forceinline__ uint2 e4m3_8(const uint4& v, float inv) {
+  uint2 r;
+  r.x = e4m3_pair(v.x, inv) | (e4m3_pair(v.y, inv) << 16);
+  r.y = e4m3_pair(v.z, inv) | (e4m3_pair(v.w, inv) << 16);
+  return r;
+}
+
+__device__ __forceinline__ uint32_t e2m1_4(const uint2& w, float inv) {
+  // 4 bf16 -> 4 E2M1 codes packed in 16 bits (element 0 in the low nibble)
+  uint32_t b0 = cvt_e2m1x2(__fmul_rn(bf16hi(w.x), inv), __fmul_rn(bf16lo(w.x), inv));
+  uint32_t b1 = cvt_e2m1x2(__fmul_rn(bf16hi(w.y), inv), __fmul_rn(bf16lo(w.y), inv));
+  return b0 | (b1 << 8);
+}
+
+__device__ __forceinline__ uint4 ld_nc(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// ------------------------------------------------------ FP8 per-token quant
+
+// A team of T threads handles one row; 256 / T rows per CTA iteration.  Up to
+// VPL 16-byte vectors per thread stay in registers between the amax and the
+// cast; longer rows re-read the remainder (L2-resident by then).
+template <int T, int VPL>
+__global__ void __launch_bounds__(256) quant_fp8_rows_kernel(const __nv_bfloat16* __restrict__ x,
+                                                             int64_t M, int64_t K, int64_t ldx,
+                                                             uint8_t* __restrict__ q,
+                                                             float* __restrict__ s, RowMap map) {
+  constexpr int TEAMS = 256 / T;
+  constexpr int WPT = T / 32;  // warps per team
+  __shared__ uint32_t red[8];
+  const int team = threadIdx.x / T;
+  const int tt = threadIdx.x % T;
+  const int64_t nvec = K >> 3;
+  for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * TEAMS; row0 < M;
+       row0 += static_cast<int64_t>(gridDim.x) * TEAMS) {
+    const int64_t row = row0 + team;
+    const bool valid = row < M;  // uniform across a warp (T >= 32)
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (valid ? map(row) : 0) * ldx);
+    uint4 v[VPL];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int64_t idx = tt + static_cast<int64_t>(i) * T;
+      if (valid && idx < nvec) {
+        v[i] = ld_nc(xr + idx);
+        amax = fmaxf(amax, absmax8(v[i]));
+      }
+    }
+    for (int64_t idx = tt + static_cast<int64_t>(VPL) * T; valid && idx < nvec; idx += T)
+      amax = fmaxf(amax, absmax8(ld_nc(xr + idx)));
+    // amax >= 0, so the float bit patterns order like unsigned integers
+    uint32_t a = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+    if constexpr (WPT > 1) {
+      if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+      __syncthreads();
+      uint32_t m = 0;
+#pragma unroll
+      for (int w = 0; w < WPT; ++w) m = max(m, red[team * WPT + w]);
+      a = m;
+      __syncthreads();
+    }
+    const float am = __uint_as_float(a);
+    const float scale = __fdiv_rn(am, 448.f);
+    const float inv = am > 0.f ? __fdiv_rn(448.f, am) : 0.f;
+    if (valid && tt == 0) s[row] = scale;
+    uint2* qr = reinterpret_cast<uint2*>(q + row * K);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int64_t idx = tt + static_cast<int64_t>(i) * T;
+      if (valid && idx < nvec) qr[idx] = e4m3_8(v[i], inv);
+    }
+    for (int64_t idx = tt + static_cast<int64_t>(VPL) * T; valid && idx < nvec; idx += T)
+      qr[idx] = e4m3_8(ld_nc(xr + idx), inv);
+  }
+}
+
+// ------------------------------------------------------------ tensor amax
+
+__global__ void __launch_bounds__(256) tensor_amax_kernel(const uint4* __restrict__ x,
+                                                          int64_t nvec, uint32_t* amax_bits) {
+  float m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < nvec; i += 4 * stride) {
+    uint4 a = ld_nc(x + i), b = ld_nc(x + i + stride), c = ld_nc(x + i + 2 * stride),
+          d = ld_nc(x + i + 3 * stride);
+    m0 = fmaxf(m0, absmax8(a));
+    m1 = fmaxf(m1, absmax8(b));
+    m2 = fmaxf(m2, absmax8(c));
+    m3 = fmaxf(m3, absmax8(d));
+  }
+  for (; i < nvec; i += stride) m0 = fmaxf(m0, absmax8(ld_nc(x + i)));
+  const float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+  const uint32_t a = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+  __shared__ uint32_t red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t b = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b = max(b, red[w]);
+    atomicMax(amax_bits, b);
+  }
+}
+
+// ------------------------------------------------------- NVFP4 block quant
+
+// One thread per 16-element block of a row.  Threads cover the padded
+// [ceil(M/128)*128, kchunks*4] grid of blocks so that padding scales are
+// written as zero.
+__global__ void __launch_bounds__(256) quant_nvfp4_kernel(
+    const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K, int64_t ldx,
+    uint8_t* __restrict__ q, uint8_t* __restrict__ sf, int64_t kchunks, int64_t mpad,
+    const uint32_t* __restrict__ amax_bits, float* g_out, RowMap map) {
+  const int64_t nbp = kchunks * 4;  // padded blocks per row
+  const int64_t nb = K >> 4;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t row = idx / nbp;
+  const int64_t b = idx - row * nbp;
+  if (row >= mpad) return;
+  const float A = __uint_as_float(*amax_bits);
+  const float G = __fdiv_rn(A, 2688.f);
+  const float enc = A > 0.f ? __fdiv_rn(448.f, A) : 0.f;
+  if (idx == 0 && g_out != nullptr) *g_out = G;
+  uint32_t sb = 0;
+  if (row < M && b < nb) {
+    const uint4* xp = reinterpret_cast<const uint4*>(x + map(row) * ldx + b * 16);
+    const uint4 v0 = ld_nc(xp), v1 = ld_nc(xp + 1);
+    const float amb = fmaxf(absmax8(v0), absmax8(v1));
+    sb = cvt_e4m3x2(0.f, __fmul_rn(amb, enc)) & 0xFF;
+    const float den = __fmul_rn(e4m3_to_f32(sb), G);
+    const float inv = den > 0.f ? __fdiv_rn(1.f, den) : 0.f;
+    uint2 out;
+    out.x = e2m1_4(make_uint2(v0.x, v0.y), inv) | (e2m1_4(make_uint2(v0.z, v0.w), inv) << 16);
+    out.y = e2m1_4(make_uint2(v1.x, v1.y), inv) | (e2m1_4(make_uint2(v1.z, v1.w), inv) << 16);
+    *reinterpret_cast<uint2*>(q + row * (K >> 1) + b * 8) = out;
+  }
+  sf[sf_offset(row, b, kchunks)] = static_cast<uint8_t>(sb);
+}
+
+__global__ void permute_bias_kernel(const __nv_bfloat16* __restrict__ src,
+                                    __nv_bfloat16* __restrict__ dst, int64_t N, RowMap map) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < N) dst[i] = src ? src[map(i)] : __float2bfloat16(0.f);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- launchers
+
+cudaError_t launch_quant_fp8_rows(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
+                                  float* s, RowMap map, int num_sms, cudaStream_t st) {
+  if (M <= 0) return cudaSuccess;
+  constexpr int VPL = 12;  // 96 bf16 per thread in registers
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  auto grid_for = [&](int teams) {
+    int64_t blocks = (M + teams - 1) / teams;
+    int64_t cap = static_cast<int64_t>(num_sms) * 8;
+    return static_cast<unsigned>(blocks < cap ? blocks : cap);
+  };
+  const int64_t per_warp = 32 * VPL * 8;
+  if (K <= per_warp) {
+    quant_fp8_rows_kernel<32, VPL><<<grid_for(8), 256, 0, st>>>(xb, M, K, ldx, q, s, map);
+  } else if (K <= 2 * per_warp) {
+    quant_fp8_rows_kernel<64, VPL><<<grid_for(4), 256, 0, st>>>(xb, M, K, ldx, q, s, map);
+  } else if (K <= 4 * per_warp) {
+    quant_fp8_rows_kernel<128, VPL><<<grid_for(2), 256, 0, st>>>(xb, M, K, ldx, q, s, map);
+  } else {
+    quant_fp8_rows_kernel<256, VPL><<<grid_for(1), 256, 0, st>>>(xb, M, K, ldx, q, s, map);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tensor_amax(const void* x, int64_t n_elems, uint32_t* amax_bits, int num_sms,
+                               cudaStream_t st) {
+  if (n_elems <= 0) return cudaSuccess;
+  const int64_t nvec = n_elems >> 3;
+  int64_t blocks = (nvec + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  tensor_amax_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      static_cast<const uint4*>(x), nvec, amax_bits);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
+                               uint8_t* sf, const uint32_t* amax_bits, float* g_out, RowMap map,
+                               cudaStream_t st) {
+  const int64_t mpad = ((M + 127) / 128) * 128;
+  const int64_t kch = sf_kchunks(K);
+  const int64_t total = mpad * kch * 4;
+  if (total <= 0) return cudaSuccess;
+  const int64_t blocks = (total + 255) / 256;
+  quant_nvfp4_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), M, K, ldx, q, sf, kch, mpad, amax_bits, g_out, map);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_bias(const void* src, void* dst, int64_t N, RowMap map,
+                                cudaStream_t st) {
+  if (N <= 0) return cudaSuccess;
+  permute_bias_kernel<<<static_cast<unsigned>((N + 255) / 256), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(src), static_cast<__nv_bfloat16*>(dst), N, map);
+  return cudaGetLastError();
+}
+
+}  // namespace qlb

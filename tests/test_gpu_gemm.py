@@ -1,0 +1,85 @@
+"""GPU parity of the whole path (quantize -> tcgen05 GEMM -> fused epilogue)
+against the oracle, element by element, within
+|gpu - ref| <= 8e-3 |ref| + 1e-3 rms(ref)  (ref = binary64, before bf16)."""
+import numpy as np
+import pytest
+
+import oracle
+from qlutil import assert_close, from_dev_bf16, sample_rows, to_dev_bf16
+from synth.tensors import draw
+
+pytestmark = pytest.mark.gpu
+
+EPIS = ["bias", "bias_gelu", "swiglu", "bias_gated_residual", "split_bias_gelu"]
+
+
+def _run(fmt, epi, M, N, K, seed=0, x_kind="normal", bias=True, rows=None, split_col=None):
+    import torch
+    import precision_gemm_qlinear_b200 as ql
+    if x_kind == "normal":
+        x = draw("normal", (M, K), seed, "x", outlier_frac=0.01, outlier_factor=8.0)
+    else:
+        x = draw("student_t", (M, K), seed, "x", nu=3, outlier_frac=0.005, outlier_factor=20.0)
+    w = draw("normal", (N, K), seed, "w", std=0.02)
+    b = draw("normal", (N,), seed, "bias", std=0.01) if bias else None
+    Nout = N // 2 if epi == "swiglu" else N
+    sc = (split_col if split_col is not None else (N // 2) // 32 * 32) if epi == "split_bias_gelu" else 0
+    gate = res = None
+    if epi == "bias_gated_residual":
+        gate = draw("normal", (Nout,), seed, "gate", mean=1.0, std=0.1)
+        res = draw("normal", (M, Nout), seed, "residual")
+    lay = ql.QLinear(fmt, epi, to_dev_bf16(w), None if b is None else to_dev_bf16(b), split_col=sc)
+    out = lay(to_dev_bf16(x), residual=None if res is None else to_dev_bf16(res),
+              gate=None if gate is None else to_dev_bf16(gate))
+    torch.cuda.synchronize()
+    assert lay.check() == 0
+    ref = oracle.qlinear_reference(fmt, epi, x, w, bias=b, residual=res, gate=gate, split_col=sc,
+                                   rows=rows)
+    got = from_dev_bf16(out)
+    if rows is not None:
+        got = got[rows]
+    return got, ref["out"]
+
+
+@pytest.mark.parametrize("epi", EPIS)
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
+def test_small_all_epilogues(fmt, epi):
+    # 3 M tiles with a ragged tail, 2-3 N tiles, several K stages
+    K = 384 if fmt == "fp8" else 512
+    got, ref = _run(fmt, epi, 300, 768 if epi != "swiglu" else 1024, K)
+    assert_close(got, ref, f"{fmt}/{epi}")
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
+def test_tiny_config(fmt):
+    got, ref = _run(fmt, "bias_gelu", 128, 512, 256)
+    assert_close(got, ref, f"tiny {fmt}")
+
+
+@pytest.mark.parametrize("M", [1, 5, 127, 129])
+def test_ragged_m(M):
+    got, ref = _run("fp8", "bias", M, 512, 256)
+    assert_close(got, ref, f"M={M}")
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
+def test_k_tail_and_no_bias(fmt):
+    # K not a multiple of the 128-byte stage: zero-filled by TMA
+    K = 208 if fmt == "fp8" else 544
+    got, ref = _run(fmt, "bias", 200, 512, K, bias=False)
+    assert_close(got, ref, f"K tail {fmt}")
+
+
+def test_fp8_n_not_multiple_of_tile():
+    got, ref = _run("fp8", "bias_gelu", 256, 288, 256)
+    assert_close(got, ref, "N=288")
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
+def test_many_tiles_per_cta(fmt):
+    # more tiles than SMs: every CTA runs several tiles and cycles both TMEM
+    # accumulator buffers; oracle on a row sample covering every M tile
+    M, N, K = 2000, 2560, 256
+    rows = sample_rows(M, 48, seed=1)
+    got, ref = _run(fmt, "split_bias_gelu", M, N, K, x_kind="t", rows=rows, split_col=1024)
+    assert_close(got, ref, f"many tiles {fmt}")

@@ -1,0 +1,26 @@
+"""The scale-factor atom layout used by the GEMM is a bijection on the padded
+[ceil(M/128)*128, ceil(K/256)*16] block grid, so un-swizzling is exact (no GPU)."""
+import numpy as np
+import pytest
+
+from qlutil import sf_layout_offsets, sf_unswizzle
+
+
+@pytest.mark.parametrize("rows,K", [(1, 32), (128, 256), (300, 3072), (257, 544), (16896, 3072)])
+def test_sf_layout_is_a_bijection(rows, K):
+    off = sf_layout_offsets(rows, K)
+    total = ((rows + 127) // 128) * ((K + 255) // 256) * 4 * 512
+    assert off.size == total
+    assert np.array_equal(np.sort(off), np.arange(total))
+
+
+def test_sf_unswizzle_roundtrip():
+    rows, K = 300, 544
+    g = np.random.default_rng(0)
+    logical = g.integers(0, 256, (rows, K // 16), dtype=np.uint8)
+    kch = ((K + 255) // 256) * 4
+    buf = np.zeros(((rows + 127) // 128) * kch * 512, np.uint8)
+    for r in range(rows):
+        for b in range(K // 16):
+            buf[((r // 128) * kch + b // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + b % 4] = logical[r, b]
+    assert np.array_equal(sf_unswizzle(buf, rows, K), logical)
