@@ -1,0 +1,489 @@
+"""Benchmark of the quantized DiT linear layer on B200.
+
+One step = one pass of the whole path over one batch of synthetic FLUX-shaped
+input: dynamic activation quantization, block-scaled tcgen05 GEMM and fused
+epilogue, for every layer of the workload (default: the FLUX-dev QKV
+projection, FP8, M=4608 K=3072 N=9216, bias epilogue).
+
+Metric: TFLOP/s of the quantized linear layer (2*M*N*K per GEMM / step time).
+Timing: W warm-up steps, then exactly K steps between CUDA events on the
+launching stream, bracketed by barrier + synchronize; max over ranks.  Input
+sets rotate so that each step reads activations and weights that are not
+L2-resident (the rotation spans more than the 126 MB L2).
+
+Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own
+tokens (weak scaling, no data-path collective); value = all ranks' FLOPs /
+max-over-ranks time.
+
+--impl reference times the CPU oracle (the reference arm of this method) on
+the host cores, on a bounded row sample per step.
+"""
+import argparse
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import WORKLOADS, make_inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = "flux_qkv_fp8"
+L2_BYTES = 126 * 2 ** 20
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# nominal dense tensor-core ratios to bf16 (FP8 4.5 / 2.25 PF, FP4 9 / 2.25 PF)
+NOMINAL_RATIO = {"fp8": 2.0, "nvfp4": 4.0}
+GEMM_SOURCES = ["precision_gemm_qlinear_b200/csrc/gemm.cu",
+                "precision_gemm_qlinear_b200/csrc/ptx.cuh",
+                "precision_gemm_qlinear_b200/csrc/internal.h"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--sets", type=int, default=0, help="input rotation sets (0 = auto)")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def gemm_source_sha():
+    h = hashlib.sha256()
+    for p in GEMM_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload, kernel_fmt):
+    """DRAM bytes per launch of the GEMM from the committed ncu summary, if the
+    kernel source has not changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("source_sha") != gemm_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index, period=0.02):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.ok = False
+        self.period = period
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        reasons = [k for k, v in self.REASONS.items() if self.reasons & v and k != "gpu_idle"]
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------- ours
+
+def to_dev(a, dev):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+class Model:
+    """The workload's layers with NSETS rotated copies of inputs and weights."""
+
+    def __init__(self, wl, dev, seed, nsets):
+        import torch
+        import precision_gemm_qlinear_b200 as ql
+        self.wl, self.dev = wl, dev
+        self.sets = []
+        host0 = None
+        for s in range(nsets):
+            layers = []
+            for li, layer in enumerate(wl.layers):
+                inp = make_inputs(layer, seed=seed * 1000 + s, layer_index=li)
+                if s == 0 and li == 0:
+                    host0 = inp
+                lay = ql.QLinear(layer.fmt, layer.epi, to_dev(inp["w"], dev),
+                                 None if inp["bias"] is None else to_dev(inp["bias"], dev),
+                                 split_col=layer.split_col)
+                codes, scales = lay.act_buffers(layer.M, dev)
+                d = dict(lay=lay, codes=codes, scales=scales,
+                         out=torch.empty((layer.M, lay.Nout), dtype=torch.bfloat16, device=dev))
+                if "x" in inp:
+                    d["x"] = to_dev(inp["x"], dev)
+                if layer.epi == "bias_gated_residual":
+                    d["gate"] = to_dev(inp["gate"], dev)
+                    d["residual"] = to_dev(inp["residual"], dev)
+                layers.append(d)
+            self.sets.append(layers)
+        self.host0 = host0
+        torch.cuda.synchronize()
+
+    def step(self, s, stream, gemm_events=None):
+        """Enqueue one pass of the path over input set s."""
+        layers = self.sets[s % len(self.sets)]
+        x = layers[0]["x"]
+        for i, d in enumerate(layers):
+            lay = d["lay"]
+            lay.quantize(x, d["codes"], d["scales"], stream)
+            if gemm_events is not None:
+                gemm_events[i][0].record(stream)
+            lay.forward_codes(d["codes"], d["scales"], x.shape[0], d["out"], d.get("residual"),
+                              d.get("gate"), stream)
+            if gemm_events is not None:
+                gemm_events[i][1].record(stream)
+            x = d["out"]
+        return x
+
+    def launches_per_step(self):
+        n = 0
+        for layer in self.wl.layers:
+            n += 2 if layer.fmt == "fp8" else 3
+        return n
+
+
+def cpu_baseline(wl, seconds):
+    """Time the oracle (as it stands) on a bounded row sample of the workload's
+    first layer; returns TFLOP/s-equivalent and a description."""
+    import oracle
+    layer = wl.layers[0]
+    inp = make_inputs(layer, seed=0)
+    x = inp.get("x")
+    if x is None:  # chained input: use a synthetic bf16 stand-in of the same shape
+        x = make_inputs(wl.layers[0], seed=0)["x"]
+    # weights quantized once, untimed (not part of the per-step path)
+    if layer.fmt == "fp8":
+        qw, sw = oracle.quant_fp8_rows(inp["w"])
+    else:
+        qw, sfw, gw = oracle.quant_nvfp4(inp["w"])
+        amax = oracle.tensor_amax(x)
+
+    def run(rows):
+        t0 = time.perf_counter()
+        xs = x[:rows]
+        if layer.fmt == "fp8":
+            qa, sa = oracle.quant_fp8_rows(xs)
+            y = oracle.gemm_fp8(qa, sa, qw, sw)
+        else:
+            qa, sfa, ga = oracle.quant_nvfp4(xs, amax=amax)
+            y = oracle.gemm_nvfp4(qa, sfa, ga, qw, sfw, gw)
+        oracle.epilogue(layer.epi, y, bias=inp["bias"], residual=inp.get("residual"),
+                        gate=inp.get("gate"), split_col=layer.split_col)
+        return time.perf_counter() - t0
+
+    probe = 2
+    t = run(probe)
+    rows = int(max(1, min(layer.M, probe * seconds / max(t, 1e-6))))
+    dt = run(rows)
+    flops = 2.0 * rows * layer.N * layer.K
+    return flops / dt / 1e12, rows, dt, oracle.num_threads()
+
+
+def main_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    rank, local_rank, world = dist_env()
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[args.workload]
+
+    per_set = 0
+    for layer in wl.layers:
+        kb = layer.K if layer.fmt == "fp8" else layer.K // 2
+        per_set += layer.M * layer.K * 2 + layer.N * kb + layer.M * (
+            layer.N // 2 if layer.epi == "swiglu" else layer.N) * 2
+    nsets = args.sets or max(2, int(np.ceil(2 * L2_BYTES / per_set)) + 1)
+    model = Model(wl, dev, seed=rank, nsets=nsets)
+    stream = torch.cuda.Stream(device=dev)
+    flops_step = float(wl.flops)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            model.step(i, stream)
+    stream.synchronize()
+    for s in model.sets:
+        for d in s:
+            st = d["lay"].check(stream)
+            if st != 0:
+                raise RuntimeError(f"device error during warm-up: status {st}")
+
+    nl = len(wl.layers)
+    gev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(nl)] for _ in range(args.steps)]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    with sampler:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for i in range(args.steps):
+                model.step(args.warmup + i, stream,
+                           gemm_events=[list(gev[i][j]) for j in range(nl)])
+            ev1.record(stream)
+        stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    total_ms = ev0.elapsed_time(ev1)
+    gemm_ms = [sum(gev[i][j][0].elapsed_time(gev[i][j][1]) for i in range(args.steps)) / args.steps
+               for j in range(nl)]
+    for s in model.sets:
+        for d in s:
+            st = d["lay"].check(stream)
+            if st != 0:
+                raise RuntimeError(f"device error during timing: status {st}")
+
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    ms_per_step = max_ms / args.steps
+    value = flops_step * world * args.steps / (max_ms / 1e3) / 1e12
+
+    # dominant kernel: the GEMM with the largest time share
+    j = int(np.argmax(gemm_ms))
+    layer = wl.layers[j]
+    peaks, peak_src = load_peaks()
+    sustained = total_ms > 1000.0
+    bf16 = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    peak = bf16 * NOMINAL_RATIO[layer.fmt]
+    achieved = layer.flops / (gemm_ms[j] / 1e3) / 1e12
+    traffic = profiled_traffic(args.workload, layer.fmt)
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                "kernel": f"qgemm_kernel<{layer.fmt},{layer.epi}>",
+                "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} x "
+                               f"{NOMINAL_RATIO[layer.fmt]:g} (nominal {layer.fmt}/bf16 ratio)",
+                "gemm_ms": round(gemm_ms[j], 5),
+                "gemm_share": round(sum(gemm_ms) / ms_per_step, 4)}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(model, stream, dev, args, world, flops_step)
+
+    cpu = None
+    if not args.no_cpu and world == 1 and rank == 0:
+        v, rows, dt, cores = cpu_baseline(wl, args.cpu_seconds)
+        cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"{rows} of {wl.layers[0].M} rows of layer 0 ({wl.layers[0].fmt} "
+                         f"{wl.layers[0].M}x{wl.layers[0].K}x{wl.layers[0].N}), quantize+GEMM+"
+                         f"epilogue, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": "quantized DiT linear TFLOP/s at FLUX shapes",
+            "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": wl.layers[0].fmt if len(set(l.fmt for l in wl.layers)) == 1 else "mixed",
+            "data": "synthetic (seeded FLUX-shaped activations and random-init weights)",
+            "config": {"workload": wl.name, "desc": wl.note,
+                       "layers": [dict(fmt=l.fmt, M=l.M, K=l.K, N=l.N, epi=l.epi) for l in wl.layers],
+                       "global_tokens": wl.layers[0].M * world, "parallelism": f"replicas{world}",
+                       "l2": f"inputs rotate over {nsets} sets ({per_set / 2**20:.0f} MB each); "
+                             "no set is L2-resident when reused"},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": model.launches_per_step() * args.steps,
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(model, stream, dev, args, world, flops_step):
+    """Same metric through the public API with host buffers: pinned-host
+    activations copied in, quantize + GEMM + epilogue, result copied out."""
+    import torch
+    wl = model.wl
+    layer0 = wl.layers[0]
+    d0 = model.sets[0][0]
+    x_host = torch.from_numpy(np.ascontiguousarray(model.host0["x"]).view(np.int16)) \
+        .view(torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(d0["x"])
+    last = model.sets[0][-1]
+    out_host = torch.empty(tuple(last["out"].shape), dtype=torch.bfloat16).pin_memory()
+    steps = max(3, min(args.steps, 50))
+    with torch.cuda.stream(stream):
+        def one():
+            x_dev.copy_(x_host, non_blocking=True)
+            x = x_dev
+            for d in model.sets[0]:
+                lay = d["lay"]
+                lay.quantize(x, d["codes"], d["scales"], stream)
+                lay.forward_codes(d["codes"], d["scales"], x.shape[0], d["out"],
+                                  d.get("residual"), d.get("gate"), stream)
+                x = d["out"]
+            out_host.copy_(x, non_blocking=True)
+        for _ in range(3):
+            one()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            one()
+        e1.record(stream)
+        stream.synchronize()
+    ms = e0.elapsed_time(e1)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    return {"value": round(flops_step * world * steps / (ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(x_host.numel() * 2),
+            "d2h_bytes_per_step": int(out_host.numel() * 2), "steps": steps}
+
+
+# ---------------------------------------------------------------- reference
+
+def main_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    wl = WORKLOADS[args.workload]
+    layer = wl.layers[0]
+    inp = make_inputs(layer, seed=0)
+    x = inp.get("x")
+    if layer.fmt == "fp8":
+        qw, sw = oracle.quant_fp8_rows(inp["w"])
+    else:
+        qw, sfw, gw = oracle.quant_nvfp4(inp["w"])
+        amax = oracle.tensor_amax(x)
+    # bounded per-step row sample so that warm-up + steps finish in a few minutes
+    per_row = 2.0 * layer.N * layer.K
+    budget_s = 150.0 / max(1, args.steps + args.warmup)
+    rows = 1
+    t0 = time.perf_counter()
+    if layer.fmt == "fp8":
+        qa, sa = oracle.quant_fp8_rows(x[:1])
+        oracle.gemm_fp8(qa, sa, qw, sw)
+    else:
+        qa, sfa, ga = oracle.quant_nvfp4(x[:1], amax=amax)
+        oracle.gemm_nvfp4(qa, sfa, ga, qw, sfw, gw)
+    t1 = time.perf_counter() - t0
+    rows = int(max(1, min(layer.M, budget_s / max(t1, 1e-6))))
+
+    def step(i):
+        r0 = (i * rows) % max(1, layer.M - rows + 1)
+        xs = x[r0:r0 + rows]
+        if layer.fmt == "fp8":
+            qa, sa = oracle.quant_fp8_rows(xs)
+            y = oracle.gemm_fp8(qa, sa, qw, sw)
+        else:
+            qa, sfa, ga = oracle.quant_nvfp4(xs, amax=amax)
+            y = oracle.gemm_nvfp4(qa, sfa, ga, qw, sfw, gw)
+        oracle.epilogue(layer.epi, y, bias=inp["bias"], split_col=layer.split_col,
+                        residual=None if "residual" not in inp else inp["residual"][r0:r0 + rows],
+                        gate=inp.get("gate"))
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = per_row * rows * args.steps / dt / 1e12
+    cores = oracle.num_threads()
+    line = {
+        "impl": "reference", "metric": "quantized DiT linear TFLOP/s at FLUX shapes",
+        "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded FLUX-shaped activations and random-init weights)",
+        "config": {"workload": wl.name, "desc": wl.note,
+                   "layers": [dict(fmt=l.fmt, M=l.M, K=l.K, N=l.N, epi=l.epi) for l in wl.layers]},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"{rows} rows of layer 0 per step (quantize + GEMM + epilogue)"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        main_reference(a)
+    else:
+        main_ours(a)
