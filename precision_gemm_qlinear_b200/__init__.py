@@ -35,12 +35,12 @@ class QLinear:
     workspace is a uint8 CUDA tensor owned by this object.
     """
 
-    def __init__(self, fmt, epi, w, bias=None, split_col=0, stream=None):
+    def __init__(self, fmt, epi, w, bias=None, split_col=0, variant=0, stream=None):
         import torch
         assert w.is_cuda and w.dtype == torch.bfloat16 and w.is_contiguous()
         N, K = w.shape
         self.fmt, self.epi, self.N, self.K = fmt, epi, int(N), int(K)
-        self.desc = make_desc(fmt, epi, N, K, split_col)
+        self.desc = make_desc(fmt, epi, N, K, split_col, variant)
         nbytes = qlinear_weight_bytes(self.desc)
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=w.device)
         self.h = qlinear_create(self.desc, w.data_ptr(), _ptr(bias), self.ws.data_ptr(), nbytes,

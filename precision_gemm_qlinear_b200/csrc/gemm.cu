@@ -1,28 +1,35 @@
 // gemm.cu -- persistent, warp-specialised tcgen05 GEMM with fused epilogue.
 //
-// One CTA per SM (persistent), 6 warps:
-//   warp 0      TMA producer: A / B operand tiles (128-byte swizzle) and, for
-//               NVFP4, the block-scale atoms (bulk copies) into an S-stage
-//               shared-memory ring guarded by full/empty mbarriers;
-//   warp 1      MMA issuer: allocates 512 TMEM columns; one elected thread
-//               issues tcgen05.mma (kind::f8f6f4 for FP8, kind::mxf4nvf4 with
-//               block16 E4M3 scales for NVFP4, scales staged to TMEM with
-//               tcgen05.cp) into a double-buffered fp32 TMEM accumulator;
-//   warps 2..5  epilogue: tcgen05.ld -> registers -> dequant scale, bias,
+// Two tile configurations share one kernel template:
+//   CG = 2 (default): a cluster of 2 CTAs (a "CTA pair" on two SMs) computes a
+//          256 x 256 tile with tcgen05.mma.cta_group::2 (M = 256).  Each CTA
+//          TMA-loads its own 128 rows of A and its own 128 rows of B (no
+//          multicast); the loads of both CTAs are counted on the leader CTA's
+//          mbarrier, and the leader's single MMA thread drives both tensor
+//          cores.  Per SM, 32 KB of operands feed 512 cycles of FP8 MMA.
+//   CG = 1: one CTA computes a 128 x 256 tile (used when M <= 128).
+// Roles (10 warps):
+//   warp 0      TMA producer: A / B tiles (128-byte swizzle) and, for NVFP4,
+//               the block-scale atoms, into an S-stage shared-memory ring
+//               guarded by full/empty mbarriers;
+//   warp 1      TMEM allocation (512 columns) and, in the leader CTA, the MMA
+//               issuer (kind::f8f6f4 for FP8; kind::mxf4nvf4 with block16 E4M3
+//               scales for NVFP4, scales staged to TMEM with tcgen05.cp) into a
+//               double-buffered fp32 TMEM accumulator;
+//   warps 2..9  epilogue: tcgen05.ld -> registers -> dequant scale, bias,
 //               activation / gated residual -> bf16 -> swizzled shared staging
-//               -> TMA store.  Each warp owns the 32 TMEM lanes (= tile rows)
-//               of its sub-partition.
-// Tile 128 x 256 x (128 bytes of K per stage); tiles are visited in groups of
-// `group_m` M-tiles for L2 reuse.  Every mbarrier wait is bounded (about one
-// second of %globaltimer); on expiry the CTA records an error code, drains
-// what it issued and exits cleanly (no trap).
+//               -> TMA store.  Two warps share each TMEM sub-partition (32
+//               rows) and split its 256 columns.
+// Tiles are visited in groups of `group_m` M-tiles for L2 reuse.  Every
+// mbarrier wait is bounded (one second of %globaltimer); on expiry the CTA
+// records an error code, drains what it issued and exits cleanly (no trap).
 //
 // The method: quantized GEMM with fused epilogues (algoritmulzilei.ro,
 // "Accelerarea generarii de imagini cu FLUX 3 Image Klein": GEMMs with fused
 // epilogues incl. SwiGLU; wavespeed.ai "Cuantizacion Dinamica FP8": the
-// matmul runs on the 8-bit tensor cores).  The pages name the Blackwell
-// features this uses (TMEM, 5th-generation tensor cores with FP8/FP4) in
-// wavespeed.ai "Arquitectura de GPU Blackwell de NVIDIA: B200".
+// matmul runs on the 8-bit tensor cores).  wavespeed.ai "Arquitectura de GPU
+// Blackwell de NVIDIA: B200" names the features used here: TMEM, CTA pairs
+// that share tensor-core work, 5th-generation tensor cores with FP8/FP4.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -35,15 +42,13 @@ namespace qlb {
 
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BM = 128;                // rows of the tile per CTA
+constexpr int BN = 256;                // columns of the tile (MMA N)
 constexpr int BK_BYTES = 128;          // K bytes per pipeline stage
 constexpr int A_BYTES = BM * BK_BYTES;  // 16 KB
-constexpr int B_BYTES = BN * BK_BYTES;  // 32 KB
-constexpr int SFA_BYTES = 2048;         // 4 atoms (one per MMA K step)
-constexpr int SFB_BYTES = 4096;         // 2 row blocks x 4 atoms
-constexpr int NUM_THREADS = 192;
-constexpr int STAGING_BYTES = 32 * 64;  // one 32 x 32 bf16 box per epilogue warp
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+constexpr int STAGING_BYTES = 32 * 64;  // one 32 x 32 bf16 box
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // 1 s
 
 // Instruction descriptors (PTX ISA, "Instruction descriptor" of tcgen05.mma):
@@ -53,26 +58,38 @@ constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // 1 s
 //  kind::mxf4nvf4: [4,6) B scale id, [7,10) A fmt (1 = E2M1), [10,13) B fmt,
 //                 [17,23) N>>3, [23] scale type (0 = UE4M3), [24,29) M>>4,
 //                 [29,31) A scale id, [31] K size (0 = 64).
-constexpr uint32_t IDESC_F8 = (1u << 4) | (0u << 7) | (0u << 10) | ((BN >> 3) << 17) |
-                              ((BM >> 4) << 24);
-constexpr uint32_t IDESC_F4 = (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | ((BM >> 4) << 24);
+template <int CG>
+constexpr uint32_t idesc_f8() {
+  return (1u << 4) | (0u << 7) | (0u << 10) | ((BN >> 3) << 17) | (((BM * CG) >> 4) << 24);
+}
+template <int CG>
+constexpr uint32_t idesc_f4() {
+  return (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | (((BM * CG) >> 4) << 24);
+}
 
-template <int FMT>
+template <int FMT, int CG>
 struct Cfg {
   static constexpr bool NV = (FMT == 1);
-  static constexpr int STAGES = NV ? 4 : 4;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + (NV ? SFA_BYTES + SFB_BYTES : 0);
+  static constexpr bool PAIR = (CG == 2);
+  static constexpr int B_BYTES = (BN / CG) * BK_BYTES;  // this CTA's rows of B
+  static constexpr int SFA_BYTES = NV ? 2048 : 0;       // 4 atoms (one per MMA K step)
+  static constexpr int SFB_BYTES = NV ? 16384 : 0;      // 4 replicated 4 KB chunks (all 256 B rows)
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = NV ? (PAIR ? 4 : 3) : (PAIR ? 6 : 4);
   static constexpr int NBUF = NV ? 1 : 2;  // staging buffers per epilogue warp
   static constexpr int STAGING_OFF = STAGES * STAGE_BYTES;
-  static constexpr int BAR_OFF = STAGING_OFF + 4 * NBUF * STAGING_BYTES;
+  static constexpr int BAR_OFF = STAGING_OFF + NUM_EPI_WARPS * NBUF * STAGING_BYTES;
+  static_assert(BAR_OFF + 256 + 1024 <= 232448, "shared memory budget");
   static constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
   // TMEM columns: FP8 -> two disjoint 256-column accumulators.
   // NVFP4 -> accumulators at 0 and 192 (overlapping in [192,256)); the scale
-  // factors of the current stage live in [448, 496).
+  // factors of the current stage live in [448, 496): A in 4 x 4 columns, B in
+  // 4 x 8 columns (one group per 64-element MMA step).
   static constexpr uint32_t ACC1 = NV ? 192 : 256;
   static constexpr uint32_t SFA_COL = 448;
   static constexpr uint32_t SFB_COL = 464;
   static constexpr bool OVL = NV;
+  static constexpr uint32_t EPI_ARRIVALS = NUM_EPI_WARPS * CG;  // per tile, at the leader
 };
 
 struct SmemBars {
@@ -146,15 +163,30 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* p, float (&o)[
   }
 }
 
-template <int FMT, int EPI>
+__device__ __forceinline__ void load_f32x32(const float* p, float (&o)[32]) {
+  const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float4 v = __ldg(q + i);
+    o[4 * i] = v.x;
+    o[4 * i + 1] = v.y;
+    o[4 * i + 2] = v.z;
+    o[4 * i + 3] = v.w;
+  }
+}
+
+template <int FMT, int EPI, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_constant__ GemmParams p) {
-  using C = Cfg<FMT>;
+  using C = Cfg<FMT, CG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   SmemBars* sb = reinterpret_cast<SmemBars*>(smem + C::BAR_OFF);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = C::PAIR ? cluster_ctarank() : 0u;  // 0 = leader of the pair
+  const int unit = C::PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int nunits = C::PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   const int num_tiles = p.tiles_m * p.tiles_n;
 
   if (threadIdx.x == 0) {
@@ -164,20 +196,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&sb->acc_full[b]), 1);
-      mbar_init(smem_u32(&sb->acc_empty[b]), 4);
+      mbar_init(smem_u32(&sb->acc_empty[b]), C::EPI_ARRIVALS);
     }
-    mbar_init(smem_u32(&sb->ovl_free), 4);
+    mbar_init(smem_u32(&sb->ovl_free), C::EPI_ARRIVALS);
     mbar_init(smem_u32(&sb->drain), 1);
     sb->abort_flag = 0;
     fence_mbarrier_init();
     fence_proxy_async_smem();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&sb->tmem_base), 512);
-    tmem_relinquish();
+    if constexpr (C::PAIR) {
+      tmem_alloc_pair(smem_u32(&sb->tmem_base), 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(&sb->tmem_base), 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (C::PAIR)
+    cluster_sync_all();  // peer barriers are initialised before any remote arrive
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sb->tmem_base;
 
@@ -191,9 +231,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
       uint32_t issued_mask = 0, issued_phase = 0;
       bool ok = true;
       bool skipped = false;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int t = unit; t < num_tiles && ok; t += nunits) {
         int mb, nb;
         tile_coords(t, p, mb, nb);
+        const int a_row = mb * (BM * CG) + static_cast<int>(rank) * BM;
+        const int b_row = nb * BN + static_cast<int>(rank) * (BN / CG);
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!wait_bar(&sb->empty[stage], phase ^ 1, sb, p.err, ERR_WAIT_PRODUCER)) {
             ok = false;
@@ -201,25 +243,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
           }
           const uint32_t fb = smem_u32(&sb->full[stage]);
           uint8_t* st = smem + stage * C::STAGE_BYTES;
-          // test hook: CTA 0 never fills its first stage, so the consumer's
-          // bounded wait must expire
+          // test hook: the leader never fills its first stage, so the MMA
+          // thread's bounded wait must expire
           const bool skip = (p.fault_mode == 1 && blockIdx.x == 0 && !skipped);
           if (skip) {
             skipped = true;
           } else {
-            mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-            tma_load_2d(smem_u32(st), &p.tmA, fb, kb * BK_BYTES, mb * BM);
-            tma_load_2d(smem_u32(st + A_BYTES), &p.tmB, fb, kb * BK_BYTES, nb * BN);
-            if constexpr (C::NV) {
-              const uint8_t* sfa = p.sfa + (static_cast<int64_t>(mb) * p.sf_kchunks_a + kb * 4) * 512;
-              const uint8_t* sfb0 =
-                  p.sfb + (static_cast<int64_t>(2 * nb) * p.sf_kchunks_b + kb * 4) * 512;
-              const uint8_t* sfb1 =
-                  p.sfb + (static_cast<int64_t>(2 * nb + 1) * p.sf_kchunks_b + kb * 4) * 512;
-              const uint32_t sfs = smem_u32(st + A_BYTES + B_BYTES);
-              bulk_load(sfs, sfa, SFA_BYTES, fb);
-              bulk_load(sfs + SFA_BYTES, sfb0, 2048, fb);
-              bulk_load(sfs + SFA_BYTES + 2048, sfb1, 2048, fb);
+            if constexpr (C::PAIR) {
+              const uint32_t lfb = mapa_shared(fb, 0);  // the leader's full barrier
+              if (rank == 0) mbar_arrive_expect_tx(fb, 2 * C::STAGE_BYTES);
+              tma_load_2d_pair(smem_u32(st), &p.tmA, lfb, kb * BK_BYTES, a_row);
+              tma_load_2d_pair(smem_u32(st + A_BYTES), &p.tmB, lfb, kb * BK_BYTES, b_row);
+              if constexpr (C::NV) {
+                // scales through 2-D maps of 2048-byte rows (uint64 x 256): the
+                // A atoms of this CTA's 128 rows (one row of the map) and the
+                // replicated B chunks of all 256 columns of the tile (8 rows;
+                // both CTAs need them)
+                const uint32_t sfs = smem_u32(st + A_BYTES + C::B_BYTES);
+                const int ka = p.sf_kchunks_a >> 2;
+                tma_load_2d_pair(sfs, &p.tmSFA, lfb, 0, (mb * 2 + static_cast<int>(rank)) * ka + kb);
+                tma_load_2d_pair(sfs + C::SFA_BYTES, &p.tmSFB, lfb, 0,
+                                 8 * (nb * p.sfb_nstages + kb));
+              }
+            } else {
+              mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+              tma_load_2d(smem_u32(st), &p.tmA, fb, kb * BK_BYTES, a_row);
+              tma_load_2d(smem_u32(st + A_BYTES), &p.tmB, fb, kb * BK_BYTES, b_row);
+              if constexpr (C::NV) {
+                const uint8_t* sfa =
+                    p.sfa + (static_cast<int64_t>(mb) * p.sf_kchunks_a + kb * 4) * 512;
+                const uint8_t* sfb =
+                    p.sfb + (static_cast<int64_t>(nb) * p.sfb_nstages + kb) * C::SFB_BYTES;
+                const uint32_t sfs = smem_u32(st + A_BYTES + C::B_BYTES);
+                bulk_load(sfs, sfa, C::SFA_BYTES, fb);
+                bulk_load(sfs + C::SFA_BYTES, sfb, C::SFB_BYTES, fb);
+              }
             }
             issued_mask |= 1u << stage;
             issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -230,8 +288,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
           }
         }
       }
-      if (sb->abort_flag) {
-        // let every load this thread issued land before the CTA exits
+      if (sb->abort_flag && rank == 0) {
+        // let every load counted on this CTA's full barriers land before exit
         for (int s = 0; s < C::STAGES; ++s)
           if (issued_mask & (1u << s)) {
             const uint32_t a = smem_u32(&sb->full[s]);
@@ -243,14 +301,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------- MMA issuer (leader only)
+    if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       bool any = false;
       int local = 0;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
+      for (int t = unit; t < num_tiles && ok; t += nunits, ++local) {
         const int buf = local & 1;
         const uint32_t use = static_cast<uint32_t>(local >> 1);
         if (!wait_bar(&sb->acc_empty[buf], (use & 1) ^ 1, sb, p.err, ERR_WAIT_MMA)) break;
@@ -270,14 +328,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
           const uint32_t a_addr = smem_u32(st);
           const uint32_t b_addr = smem_u32(st + A_BYTES);
           if constexpr (C::NV) {
-            const uint32_t sfs = smem_u32(st + A_BYTES + B_BYTES);
+            const uint32_t sfs = smem_u32(st + A_BYTES + C::B_BYTES);
+            // per MMA step j: the A atom (32 x 128-bit, replicated to the 4
+            // sub-partitions by the copy) and the pre-replicated B chunk
+            // (128 x 256-bit)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              tc_cp_32x128b_warpx4(tmem + C::SFA_COL + 4 * j, sdesc_k_interleave(sfs + 512 * j));
-              tc_cp_32x128b_warpx4(tmem + C::SFB_COL + 8 * j,
-                                   sdesc_k_interleave(sfs + SFA_BYTES + 512 * j));
-              tc_cp_32x128b_warpx4(tmem + C::SFB_COL + 8 * j + 4,
-                                   sdesc_k_interleave(sfs + SFA_BYTES + 2048 + 512 * j));
+              const uint64_t da = sdesc_k_interleave(sfs + 512 * j);
+              const uint64_t db = sdesc_k_interleave2(sfs + C::SFA_BYTES + 4096 * j, 128, 256);
+              if constexpr (C::PAIR) {
+                tc_cp_32x128b_warpx4_pair(tmem + C::SFA_COL + 4 * j, da);
+                tc_cp_128x256b_pair(tmem + C::SFB_COL + 8 * j, db);
+              } else {
+                tc_cp_32x128b_warpx4(tmem + C::SFA_COL + 4 * j, da);
+                tc_cp_128x256b(tmem + C::SFB_COL + 8 * j, db);
+              }
             }
           }
 #pragma unroll
@@ -285,25 +350,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
             const uint64_t ad = sdesc_k_sw128(a_addr + 32 * j);
             const uint64_t bd = sdesc_k_sw128(b_addr + 32 * j);
             const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
-            if constexpr (C::NV)
-              mma_mxf4nvf4(d_tmem, ad, bd, IDESC_F4, tmem + C::SFA_COL + 4 * j,
-                           tmem + C::SFB_COL + 8 * j, acc);
-            else
-              mma_f8f6f4(d_tmem, ad, bd, IDESC_F8, acc);
+            if constexpr (C::NV) {
+              if constexpr (C::PAIR)
+                mma_mxf4nvf4_pair(d_tmem, ad, bd, idesc_f4<CG>(), tmem + C::SFA_COL + 4 * j,
+                                  tmem + C::SFB_COL + 8 * j, acc);
+              else
+                mma_mxf4nvf4(d_tmem, ad, bd, idesc_f4<CG>(), tmem + C::SFA_COL + 4 * j,
+                             tmem + C::SFB_COL + 8 * j, acc);
+            } else {
+              if constexpr (C::PAIR)
+                mma_f8f6f4_pair(d_tmem, ad, bd, idesc_f8<CG>(), acc);
+              else
+                mma_f8f6f4(d_tmem, ad, bd, idesc_f8<CG>(), acc);
+            }
           }
           any = true;
-          tc_commit(smem_u32(&sb->empty[stage]));
+          if constexpr (C::PAIR)
+            tc_commit_pair_mc(smem_u32(&sb->empty[stage]), 0x3);
+          else
+            tc_commit(smem_u32(&sb->empty[stage]));
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        tc_commit(smem_u32(&sb->acc_full[buf]));
+        if constexpr (C::PAIR)
+          tc_commit_pair_mc(smem_u32(&sb->acc_full[buf]), 0x3);
+        else
+          tc_commit(smem_u32(&sb->acc_full[buf]));
       }
       if (sb->abort_flag && any) {
         // no MMA may still be writing TMEM when it is released
-        tc_commit(smem_u32(&sb->drain));
+        if constexpr (C::PAIR)
+          tc_commit_pair_mc(smem_u32(&sb->drain), 0x1);
+        else
+          tc_commit(smem_u32(&sb->drain));
         const uint32_t a = smem_u32(&sb->drain);
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
@@ -312,21 +394,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
     }
   } else {
     // --------------------------------------------------------- epilogue
-    const int sp = warp & 3;  // TMEM sub-partition = rows [32 sp, 32 sp + 32) of the tile
-    uint8_t* staging = smem + C::STAGING_OFF + (warp - 2) * C::NBUF * STAGING_BYTES;
-    constexpr int NCH = (EPI == EPI_SWIGLU) ? 4 : 8;  // output chunks of 32 columns per tile
+    const int ew = warp - 2;           // 0..7
+    const int sp = warp & 3;           // TMEM sub-partition: rows [32 sp, 32 sp + 32) of the CTA tile
+    const int half = ew >> 2;          // which half of the tile's columns this warp owns
+    uint8_t* staging = smem + C::STAGING_OFF + ew * C::NBUF * STAGING_BYTES;
+    constexpr int NCH = (EPI == EPI_SWIGLU) ? 2 : 4;  // 32-column output chunks per warp per tile
+    const uint32_t ovl_l0 = mapa_shared(smem_u32(&sb->ovl_free), 0);
     int local = 0;
     uint32_t nstore = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
+    for (int t = unit; t < num_tiles; t += nunits, ++local) {
       int mb, nb;
       tile_coords(t, p, mb, nb);
       const int buf = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
       if (!wait_bar(&sb->acc_full[buf], use & 1, sb, p.err, ERR_WAIT_EPI)) break;
       tc_fence_after();
-      const int m = mb * BM + sp * 32 + lane;
+      // NVFP4: the accumulator columns shared by the two TMEM buffers belong to
+      // half 1 of buffer 0 and half 0 of buffer 1; those warps read them first
+      // and then release the overlap so the next tile's MMA can start.
+      const bool ovl_owner = C::OVL && (half == (buf == 0 ? 1 : 0));
+      if (C::OVL && !ovl_owner) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(ovl_l0);
+      }
+      const int row0 = mb * (BM * CG) + static_cast<int>(rank) * BM + sp * 32;  // first row of this warp
+      const int m = row0 + lane;
       const bool row_ok = m < p.M;
-      const bool slab_ok = (mb * BM + sp * 32) < p.M;
+      const bool slab_ok = row0 < p.M;
       float rs;
       if constexpr (C::NV)
         rs = __ldg(p.ga) * __ldg(p.gw);
@@ -334,24 +428,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
         rs = row_ok ? __ldg(p.sa + m) : 0.f;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(sp * 32) << 16) + (buf ? C::ACC1 : 0u);
       for (int ci = 0; ci < NCH; ++ci) {
-        const int c = (C::OVL && buf == 0) ? (ci + NCH - 2) % NCH : ci;
+        const int lc = (ovl_owner && buf == 0) ? (ci + 2) % NCH : ci;
+        const int c = half * NCH + lc;  // chunk index within the tile (output chunks for SwiGLU)
         uint32_t ra[32];
         tmem_ld_32x32b_x32(tbase + 32 * c, ra);
         uint32_t rb[32];
         if constexpr (EPI == EPI_SWIGLU) tmem_ld_32x32b_x32(tbase + 128 + 32 * c, rb);
         tmem_wait_ld();
-        if (C::OVL && ci == 1) {
+        if (ovl_owner && ci == 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&sb->ovl_free));
+          if (lane == 0) mbar_arrive_cluster(ovl_l0);
         }
         if (ci == NCH - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&sb->acc_empty[buf]));
+          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sb->acc_empty[buf]), 0));
         }
         // ---- epilogue math on 32 columns of this thread's row
-        const int ncol = nb * BN + 32 * c;                          // GEMM column of ra[0]
+        const int ncol = nb * BN + 32 * c;                                     // GEMM column of ra[0]
         const int ocol = (EPI == EPI_SWIGLU) ? nb * (BN / 2) + 32 * c : ncol;  // output column
         if (ncol >= p.N) continue;  // past the last column (N % 32 == 0); warp-uniform
         uint32_t packed[16];
@@ -362,38 +457,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
           load_bf16x32(p.bias + ncol + 128, bias_b);
           float sw_a[32], sw_b[32];
           if constexpr (!C::NV) {
-            const float4* s4a = reinterpret_cast<const float4*>(p.sw + ncol);
-            const float4* s4b = reinterpret_cast<const float4*>(p.sw + ncol + 128);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float4 a4 = __ldg(s4a + i), b4 = __ldg(s4b + i);
-              sw_a[4 * i] = a4.x; sw_a[4 * i + 1] = a4.y; sw_a[4 * i + 2] = a4.z; sw_a[4 * i + 3] = a4.w;
-              sw_b[4 * i] = b4.x; sw_b[4 * i + 1] = b4.y; sw_b[4 * i + 2] = b4.z; sw_b[4 * i + 3] = b4.w;
-            }
+            load_f32x32(p.sw + ncol, sw_a);
+            load_f32x32(p.sw + ncol + 128, sw_b);
           }
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             float o[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const float sa_ = C::NV ? rs : rs * sw_a[i + h];
-              const float sb_ = C::NV ? rs : rs * sw_b[i + h];
-              const float g = __uint_as_float(ra[i + h]) * sa_ + bias_a[i + h];
-              const float u = __uint_as_float(rb[i + h]) * sb_ + bias_b[i + h];
+              float sa_, sb_;
+              if constexpr (C::NV) {
+                sa_ = rs;
+                sb_ = rs;
+              } else {
+                sa_ = rs * sw_a[i + h];
+                sb_ = rs * sw_b[i + h];
+              }
+              const float g = fmaf(__uint_as_float(ra[i + h]), sa_, bias_a[i + h]);
+              const float u = fmaf(__uint_as_float(rb[i + h]), sb_, bias_b[i + h]);
               o[h] = silu_f(g) * u;
             }
             packed[i >> 1] = pack_bf16x2(o[0], o[1]);
           }
         } else {
           float sw_a[32];
-          if constexpr (!C::NV) {
-            const float4* s4a = reinterpret_cast<const float4*>(p.sw + ncol);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float4 a4 = __ldg(s4a + i);
-              sw_a[4 * i] = a4.x; sw_a[4 * i + 1] = a4.y; sw_a[4 * i + 2] = a4.z; sw_a[4 * i + 3] = a4.w;
-            }
-          }
+          if constexpr (!C::NV) load_f32x32(p.sw + ncol, sw_a);
           float gate_a[32], res_a[32];
           if constexpr (EPI == EPI_GATED_RES) {
             load_bf16x32(p.gate + ocol, gate_a);
@@ -404,16 +492,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
               for (int i = 0; i < 32; ++i) res_a[i] = 0.f;
             }
           }
-          const bool gelu_chunk = (EPI == EPI_BIAS_GELU) || (EPI == EPI_SPLIT && ncol >= p.split_col);
+          const bool gelu_chunk =
+              (EPI == EPI_BIAS_GELU) || (EPI == EPI_SPLIT && ncol >= p.split_col);
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
             float o[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const float s_ = C::NV ? rs : rs * sw_a[i + h];
-              float v = __uint_as_float(ra[i + h]) * s_ + bias_a[i + h];
+              float s_;
+              if constexpr (C::NV)
+                s_ = rs;
+              else
+                s_ = rs * sw_a[i + h];
+              float v = fmaf(__uint_as_float(ra[i + h]), s_, bias_a[i + h]);
               if constexpr (EPI == EPI_GATED_RES) v = fmaf(gate_a[i + h], v, res_a[i + h]);
-              if (EPI == EPI_BIAS_GELU || EPI == EPI_SPLIT) {
+              if constexpr (EPI == EPI_BIAS_GELU || EPI == EPI_SPLIT) {
                 if (gelu_chunk) v = gelu_tanh_f(v);
               }
               o[h] = v;
@@ -423,12 +516,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
         }
         // ---- stage through swizzled shared memory, then one TMA store per warp
         uint8_t* sbuf = staging + (nstore % C::NBUF) * STAGING_BYTES;
-        if (lane == 0) {
-          if constexpr (C::NBUF == 2)
-            bulk_wait_group_read<1>();
-          else
-            bulk_wait_group_read<0>();
-        }
+        if (lane == 0) bulk_wait_group_read<C::NBUF - 1>();
         __syncwarp();
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -439,7 +527,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && slab_ok) {
-          tma_store_2d(&p.tmC, smem_u32(sbuf), ocol, mb * BM + sp * 32);
+          tma_store_2d(&p.tmC, smem_u32(sbuf), ocol, row0);
           bulk_commit_group();
         }
         ++nstore;
@@ -448,36 +536,65 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
     if (lane == 0) bulk_wait_group<0>();
   }
 
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if constexpr (C::PAIR)
+    cluster_sync_all();  // no CTA leaves while its peer may still signal its barriers
+  else
+    __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    if constexpr (C::PAIR)
+      tmem_dealloc_pair(tmem, 512);
+    else
+      tmem_dealloc(tmem, 512);
   }
 }
 
-template <int FMT, int EPI>
+template <int FMT, int EPI, int CG>
 cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t st) {
-  using C = Cfg<FMT>;
+  using C = Cfg<FMT, CG>;
   static bool attr_set = false;
+  auto kern = qgemm_kernel<FMT, EPI, CG>;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(qgemm_kernel<FMT, EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int tiles = p.tiles_m * p.tiles_n;
-  const int grid = tiles < num_sms ? tiles : num_sms;
+  const int units = num_sms / CG;
+  const int grid = (tiles < units ? tiles : units) * CG;
   if (grid <= 0) return cudaSuccess;
-  qgemm_kernel<FMT, EPI><<<grid, NUM_THREADS, C::SMEM_BYTES, st>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 }  // namespace
 
-cudaError_t launch_gemm(int fmt, int epi, const GemmParams& p, int num_sms, cudaStream_t st) {
-#define QLB_CASE(F, E) \
-  if (fmt == F && epi == E) return launch_one<F, E>(p, num_sms, st);
+int gemm_smem_bytes(int fmt, int cg) {
+  if (fmt == 0) return cg == 2 ? Cfg<0, 2>::SMEM_BYTES : Cfg<0, 1>::SMEM_BYTES;
+  return cg == 2 ? Cfg<1, 2>::SMEM_BYTES : Cfg<1, 1>::SMEM_BYTES;
+}
+
+cudaError_t launch_gemm(int fmt, int epi, int cg, const GemmParams& p, int num_sms,
+                        cudaStream_t st) {
+#define QLB_CASE(F, E)                                                     \
+  if (fmt == F && epi == E) {                                              \
+    return cg == 2 ? launch_one<F, E, 2>(p, num_sms, st)                   \
+                   : launch_one<F, E, 1>(p, num_sms, st);                  \
+  }
   QLB_CASE(0, EPI_BIAS)
   QLB_CASE(0, EPI_BIAS_GELU)
   QLB_CASE(0, EPI_SWIGLU)

@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 namespace qlb {
@@ -37,15 +38,39 @@ __host__ __device__ __forceinline__ int64_t sf_bytes(int64_t rows, int64_t K) {
   return ((rows + 127) / 128) * sf_kchunks(K) * 512;
 }
 
+// Scale-factor layout of the weight (B) operand, fed to TMEM by one
+// tcgen05.cp.128x256b per 64-element MMA step: for every 256-row N tile, every
+// stage of 256 K-elements and every MMA step j (0..3) there is a 4096-byte
+// chunk of 128 rows x 32 bytes.  Row (TMEM lane) l = 32 q + r0 holds, in word
+// w (0..7), the 4 scales of weight row 256 nb + 32 w + r0 for that step --
+// the same for every q (the replication across the four TMEM sub-partitions
+// that the MMA reads).  Chunks are ordered [nb][stage][j]; the 32-byte rows
+// are stored in the unswizzled K-major core-matrix order the copy expects:
+// 8-row groups 256 bytes apart, the two 16-byte halves of a row 128 bytes
+// apart, rows of a group 16 bytes apart.
+__host__ __device__ __forceinline__ int64_t sfb_stages(int64_t K) { return (K + 255) / 256; }
+__host__ __device__ __forceinline__ int64_t sfb_bytes(int64_t rows, int64_t K) {
+  return ((rows + 255) / 256) * sfb_stages(K) * 4 * 4096;
+}
+// byte offset of the scale word of weight row n, stage ks, step j, replica q
+__host__ __device__ __forceinline__ int64_t sfb_word_offset(int64_t n, int64_t ks, int64_t j,
+                                                            int64_t q, int64_t nks) {
+  const int64_t l = q * 32 + (n & 31), w = (n & 255) >> 5;
+  return (((n >> 8) * nks + ks) * 4 + j) * 4096 + (l >> 3) * 256 + (w >> 2) * 128 + (l & 7) * 16 +
+         (w & 3) * 4;
+}
+
 // -------------------------------------------------------------- quantize
 
 cudaError_t launch_quant_fp8_rows(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
                                   float* s, RowMap map, int num_sms, cudaStream_t st);
 cudaError_t launch_tensor_amax(const void* x, int64_t n_elems, uint32_t* amax_bits, int num_sms,
                                cudaStream_t st);
+// sf_layout: 0 = activation (A operand) atoms [sf_offset], 1 = weight (B
+// operand) replicated chunks [sfb_word_offset].
 cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
-                               uint8_t* sf, const uint32_t* amax_bits, float* g_out, RowMap map,
-                               cudaStream_t st);
+                               uint8_t* sf, int sf_layout, const uint32_t* amax_bits,
+                               float* g_out, RowMap map, cudaStream_t st);
 cudaError_t launch_permute_bias(const void* src, void* dst, int64_t N, RowMap map,
                                 cudaStream_t st);
 
@@ -56,12 +81,14 @@ enum Epi : int32_t { EPI_BIAS = 0, EPI_BIAS_GELU = 1, EPI_SWIGLU = 2, EPI_GATED_
 
 struct alignas(64) GemmParams {
   CUtensorMap tmA;  // activation codes [M, K(/2)] bytes, box 128 x 128 B, 128B swizzle
-  CUtensorMap tmB;  // weight codes [N, K(/2)] bytes, box 128 B x 256 rows, 128B swizzle
+  CUtensorMap tmB;  // weight codes [N, K(/2)] bytes, box 128 B x (256 / CG) rows, 128B swizzle
   CUtensorMap tmC;  // output [M, Nout] bf16, box 32 x 32, 64B swizzle
+  CUtensorMap tmSFA;  // NVFP4 pair mode: activation SF atoms as rows of 2048 bytes
+  CUtensorMap tmSFB;  // NVFP4 pair mode: weight SF chunks as rows of 2048 bytes
   const float* sa;        // FP8: per-row activation scale [M]
   const float* sw;        // FP8: per-column weight scale [N]
-  const uint8_t* sfa;     // NVFP4: activation SF atoms
-  const uint8_t* sfb;     // NVFP4: weight SF atoms
+  const uint8_t* sfa;     // NVFP4: activation SF atoms (sf_offset layout)
+  const uint8_t* sfb;     // NVFP4: weight SF chunks (sfb_word_offset layout)
   const float* ga;        // NVFP4: activation global scale (device scalar)
   const float* gw;        // NVFP4: weight global scale (device scalar)
   const __nv_bfloat16* bias;      // [N] (zeros when the layer has no bias)
@@ -71,11 +98,14 @@ struct alignas(64) GemmParams {
   int32_t M, N, Nout, split_col;
   int32_t k_blocks;       // number of 128-byte K stages
   int32_t tiles_m, tiles_n, group_m;
-  int32_t sf_kchunks_a, sf_kchunks_b;
+  int32_t sf_kchunks_a, sfb_nstages;
   int32_t fault_mode;     // test hook: 0 = none
 };
 
-cudaError_t launch_gemm(int fmt, int epi, const GemmParams& p, int num_sms, cudaStream_t st);
+// cg = 1: one CTA per 128 x 256 tile; cg = 2: a CTA pair per 256 x 256 tile.
+cudaError_t launch_gemm(int fmt, int epi, int cg, const GemmParams& p, int num_sms,
+                        cudaStream_t st);
+int gemm_smem_bytes(int fmt, int cg);
 
 // Error codes written to the device error word by the GEMM watchdog.
 enum : uint32_t { ERR_WAIT_PRODUCER = 1u, ERR_WAIT_MMA = 2u, ERR_WAIT_EPI = 4u };

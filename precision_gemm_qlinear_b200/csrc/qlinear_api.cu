@@ -32,7 +32,9 @@ struct qlinear_s {
   uint32_t* wamax;   // NVFP4 amax word used while quantizing W
   __nv_bfloat16* bias;
   RowMap map;
-  CUtensorMap tmB;
+  CUtensorMap tmB1;    // weight codes, box 128 B x 256 rows (one CTA per tile)
+  CUtensorMap tmB2;    // weight codes, box 128 B x 128 rows (CTA pair per tile)
+  CUtensorMap tmSFB;   // NVFP4: weight SF atoms as 2048-byte rows (CTA pair)
 };
 
 namespace {
@@ -57,7 +59,7 @@ WsLayout ws_layout(const ql_desc& d) {
                                               : static_cast<size_t>(d.N) * d.K;
   off = align_up(off + code_bytes, 1024);
   L.scales = off;
-  const size_t sc_bytes = d.fmt == QL_NVFP4 ? static_cast<size_t>(sf_bytes(d.N, d.K)) + 16
+  const size_t sc_bytes = d.fmt == QL_NVFP4 ? static_cast<size_t>(sfb_bytes(d.N, d.K)) + 16
                                             : static_cast<size_t>(d.N) * 4;
   off = align_up(off + sc_bytes, 1024);
   L.bias = off;
@@ -70,7 +72,7 @@ ql_status check_desc(const ql_desc* d) {
   if (!d) return QL_ERR_INVALID_ARG;
   if (d->fmt != QL_FP8_E4M3 && d->fmt != QL_NVFP4) return QL_ERR_INVALID_ARG;
   if (d->epi < QL_EPI_BIAS || d->epi > QL_EPI_SPLIT_BIAS_GELU) return QL_ERR_INVALID_ARG;
-  if (d->flags != 0 || d->variant != 0) return QL_ERR_INVALID_ARG;
+  if (d->flags != 0 || d->variant < 0 || d->variant > 2) return QL_ERR_INVALID_ARG;
   if (d->N < 1 || d->K < 1 || d->N > (1 << 24) || d->K > (1 << 24)) return QL_ERR_INVALID_ARG;
   if (d->N % 32 != 0) return QL_ERR_INVALID_ARG;
   if (d->fmt == QL_FP8_E4M3 && d->K % 16 != 0) return QL_ERR_INVALID_ARG;
@@ -145,6 +147,14 @@ bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Scale-factor buffers viewed as rows of 2048 bytes: uint64 elements, 256 per
+// row, box = `box_rows` rows (activation atoms: 1 row = one pipeline stage of
+// one 128-row block; weight chunks: 8 rows = one stage of one 256-row tile).
+bool make_sf_tmap(CUtensorMap* m, const void* base, int64_t bytes, uint32_t box_rows) {
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, base, 256, bytes / 2048, 2048, 256,
+                   box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 ql_status from_cuda(cudaError_t e) {
@@ -227,12 +237,12 @@ ql_status qlinear_create(const ql_desc* desc, const void* w_bf16, const void* bi
                               st);
   } else if (e == cudaSuccess) {
     h->wsf = h->ws + L.scales;
-    h->wG = reinterpret_cast<float*>(h->wsf + sf_bytes(h->N, h->K));
+    h->wG = reinterpret_cast<float*>(h->wsf + sfb_bytes(h->N, h->K));
     h->wamax = reinterpret_cast<uint32_t*>(h->wG + 1);
     e = cudaMemsetAsync(h->wamax, 0, 4, st);
     if (e == cudaSuccess) e = launch_tensor_amax(w_bf16, h->N * h->K, h->wamax, h->num_sms, st);
     if (e == cudaSuccess)
-      e = launch_quant_nvfp4(w_bf16, h->N, h->K, h->K, h->wcodes, h->wsf, h->wamax, h->wG, h->map,
+      e = launch_quant_nvfp4(w_bf16, h->N, h->K, h->K, h->wcodes, h->wsf, 1, h->wamax, h->wG, h->map,
                              st);
   }
   if (e == cudaSuccess) e = launch_permute_bias(bias_bf16, h->bias, h->N, h->map, st);
@@ -242,8 +252,13 @@ ql_status qlinear_create(const ql_desc* desc, const void* w_bf16, const void* bi
     return QL_ERR_CUDA;
   }
   const uint64_t kbytes = desc->fmt == QL_NVFP4 ? h->K / 2 : h->K;
-  if (!make_tmap(&h->tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, 128, 256,
-                 CU_TENSOR_MAP_SWIZZLE_128B)) {
+  bool ok = make_tmap(&h->tmB1, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, 128,
+                      256, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            make_tmap(&h->tmB2, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, 128,
+                      128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (ok && desc->fmt == QL_NVFP4)
+    ok = make_sf_tmap(&h->tmSFB, h->wsf, sfb_bytes(h->N, h->K), 8);
+  if (!ok) {
     delete h;
     return QL_ERR_CUDA;
   }
@@ -282,7 +297,7 @@ ql_status qlinear_quantize_act(qlinear_t h, const void* x_bf16, int64_t M, void*
     e = cudaMemsetAsync(amax, 0, 4, st);
     if (e == cudaSuccess) e = launch_tensor_amax(x_bf16, M * h->K, amax, h->num_sms, st);
     if (e == cudaSuccess)
-      e = launch_quant_nvfp4(x_bf16, M, h->K, h->K, static_cast<uint8_t*>(codes), sf, amax, g,
+      e = launch_quant_nvfp4(x_bf16, M, h->K, h->K, static_cast<uint8_t*>(codes), sf, 0, amax, g,
                              RowMap{0, 0}, st);
   }
   if (e != cudaSuccess) cudaGetLastError();
@@ -304,12 +319,18 @@ ql_status qlinear_forward(qlinear_t h, const void* codes, const void* scales, in
   std::memset(&p, 0, sizeof(p));
   const bool nv = h->d.fmt == QL_NVFP4;
   const uint64_t kbytes = nv ? h->K / 2 : h->K;
+  // one CTA per 128-row tile for a single M tile, else CTA pairs on 256 rows
+  const int cg = h->d.variant == 1 ? 1 : (h->d.variant == 2 ? 2 : (M > 128 ? 2 : 1));
   if (!make_tmap(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, kbytes, M, kbytes, 128, 128,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap(&p.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out_bf16, h->Nout, M, h->Nout * 2, 32,
                  32, CU_TENSOR_MAP_SWIZZLE_64B))
     return QL_ERR_CUDA;
-  p.tmB = h->tmB;
+  p.tmB = cg == 2 ? h->tmB2 : h->tmB1;
+  if (nv && cg == 2) {
+    if (!make_sf_tmap(&p.tmSFA, scales, sf_bytes(M, h->K), 1)) return QL_ERR_CUDA;
+    p.tmSFB = h->tmSFB;
+  }
   if (nv) {
     p.sfa = static_cast<const uint8_t*>(scales);
     p.ga = reinterpret_cast<const float*>(p.sfa + sf_bytes(M, h->K));
@@ -328,13 +349,14 @@ ql_status qlinear_forward(qlinear_t h, const void* codes, const void* scales, in
   p.Nout = static_cast<int32_t>(h->Nout);
   p.split_col = static_cast<int32_t>(h->d.split_col);
   p.k_blocks = static_cast<int32_t>((kbytes + 127) / 128);
-  p.tiles_m = static_cast<int32_t>((M + 127) / 128);
+  p.tiles_m = static_cast<int32_t>((M + 128 * cg - 1) / (128 * cg));
   p.tiles_n = static_cast<int32_t>((h->N + 255) / 256);
   p.group_m = 8;
   p.sf_kchunks_a = static_cast<int32_t>(sf_kchunks(h->K));
-  p.sf_kchunks_b = static_cast<int32_t>(sf_kchunks(h->K));
+  p.sfb_nstages = static_cast<int32_t>(sfb_stages(h->K));
   p.fault_mode = 0;
-  cudaError_t e = launch_gemm(h->d.fmt, h->d.epi, p, h->num_sms, static_cast<cudaStream_t>(stream));
+  cudaError_t e =
+      launch_gemm(h->d.fmt, h->d.epi, cg, p, h->num_sms, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();
     return QL_ERR_CUDA;
@@ -369,17 +391,18 @@ ql_status qlinear_export_weights(qlinear_t h, void* codes_host, void* scales_hos
     float* sh = static_cast<float*>(scales_host);
     for (int64_t p = 0; p < h->N; ++p) sh[h->map(p)] = sc[p];
   } else {
-    std::vector<uint8_t> sf(sf_bytes(h->N, h->K));
+    std::vector<uint8_t> sf(sfb_bytes(h->N, h->K));
     float g = 0.f;
     if (cudaMemcpy(sf.data(), h->wsf, sf.size(), cudaMemcpyDeviceToHost) != cudaSuccess ||
         cudaMemcpy(&g, h->wG, 4, cudaMemcpyDeviceToHost) != cudaSuccess) {
       cudaGetLastError();
       return QL_ERR_CUDA;
     }
-    const int64_t nb = h->K / 16, kch = sf_kchunks(h->K);
+    const int64_t nb = h->K / 16, nks = sfb_stages(h->K);
     uint8_t* sh = static_cast<uint8_t*>(scales_host);
     for (int64_t p = 0; p < h->N; ++p)
-      for (int64_t b = 0; b < nb; ++b) sh[h->map(p) * nb + b] = sf[sf_offset(p, b, kch)];
+      for (int64_t b = 0; b < nb; ++b)
+        sh[h->map(p) * nb + b] = sf[sfb_word_offset(p, b / 16, (b / 4) & 3, 0, nks) + (b & 3)];
     if (global_scale) *global_scale = g;
   }
   return QL_OK;

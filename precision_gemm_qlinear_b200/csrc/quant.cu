@@ -149,37 +149,51 @@ __global__ void __launch_bounds__(256) tensor_amax_kernel(const uint4* __restric
 
 // ------------------------------------------------------- NVFP4 block quant
 
-// One thread per 16-element block of a row.  Threads cover the padded
-// [ceil(M/128)*128, kchunks*4] grid of blocks so that padding scales are
-// written as zero.
+// One thread per 64 elements (4 blocks of 16) of a row.  Threads cover the
+// padded grid [ceil(M/128)*128 rows, ceil(K/256)*4 groups] so that every
+// padding scale is written as zero.
 __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
     const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K, int64_t ldx,
-    uint8_t* __restrict__ q, uint8_t* __restrict__ sf, int64_t kchunks, int64_t mpad,
+    uint8_t* __restrict__ q, uint8_t* __restrict__ sf, int sf_layout, int64_t nks, int64_t mpad,
     const uint32_t* __restrict__ amax_bits, float* g_out, RowMap map) {
-  const int64_t nbp = kchunks * 4;  // padded blocks per row
+  const int64_t ngp = nks * 4;  // padded 64-element groups per row
   const int64_t nb = K >> 4;
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t row = idx / nbp;
-  const int64_t b = idx - row * nbp;
+  const int64_t row = idx / ngp;
+  const int64_t g = idx - row * ngp;
   if (row >= mpad) return;
   const float A = __uint_as_float(*amax_bits);
   const float G = __fdiv_rn(A, 2688.f);
   const float enc = A > 0.f ? __fdiv_rn(448.f, A) : 0.f;
   if (idx == 0 && g_out != nullptr) *g_out = G;
-  uint32_t sb = 0;
-  if (row < M && b < nb) {
-    const uint4* xp = reinterpret_cast<const uint4*>(x + map(row) * ldx + b * 16);
-    const uint4 v0 = ld_nc(xp), v1 = ld_nc(xp + 1);
-    const float amb = fmaxf(absmax8(v0), absmax8(v1));
-    sb = cvt_e4m3x2(0.f, __fmul_rn(amb, enc)) & 0xFF;
-    const float den = __fmul_rn(e4m3_to_f32(sb), G);
-    const float inv = den > 0.f ? __fdiv_rn(1.f, den) : 0.f;
-    uint2 out;
-    out.x = e2m1_4(make_uint2(v0.x, v0.y), inv) | (e2m1_4(make_uint2(v0.z, v0.w), inv) << 16);
-    out.y = e2m1_4(make_uint2(v1.x, v1.y), inv) | (e2m1_4(make_uint2(v1.z, v1.w), inv) << 16);
-    *reinterpret_cast<uint2*>(q + row * (K >> 1) + b * 8) = out;
+  uint32_t word = 0;  // the 4 block-scale codes of this group, block 4g in the low byte
+  if (row < M) {
+    const __nv_bfloat16* xr = x + map(row) * ldx;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t b = g * 4 + i;
+      if (b < nb) {
+        const uint4* xp = reinterpret_cast<const uint4*>(xr + b * 16);
+        const uint4 v0 = ld_nc(xp), v1 = ld_nc(xp + 1);
+        const float amb = fmaxf(absmax8(v0), absmax8(v1));
+        const uint32_t sb = cvt_e4m3x2(0.f, __fmul_rn(amb, enc)) & 0xFF;
+        const float den = __fmul_rn(e4m3_to_f32(sb), G);
+        const float inv = den > 0.f ? __fdiv_rn(1.f, den) : 0.f;
+        uint2 out;
+        out.x = e2m1_4(make_uint2(v0.x, v0.y), inv) | (e2m1_4(make_uint2(v0.z, v0.w), inv) << 16);
+        out.y = e2m1_4(make_uint2(v1.x, v1.y), inv) | (e2m1_4(make_uint2(v1.z, v1.w), inv) << 16);
+        *reinterpret_cast<uint2*>(q + row * (K >> 1) + b * 8) = out;
+        word |= sb << (8 * i);
+      }
+    }
   }
-  sf[sf_offset(row, b, kchunks)] = static_cast<uint8_t>(sb);
+  if (sf_layout == 0) {
+    *reinterpret_cast<uint32_t*>(sf + sf_offset(row, g * 4, nks * 4)) = word;
+  } else {
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4)
+      *reinterpret_cast<uint32_t*>(sf + sfb_word_offset(row, g >> 2, g & 3, q4, nks)) = word;
+  }
 }
 
 __global__ void permute_bias_kernel(const __nv_bfloat16* __restrict__ src,
@@ -228,15 +242,17 @@ cudaError_t launch_tensor_amax(const void* x, int64_t n_elems, uint32_t* amax_bi
 }
 
 cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
-                               uint8_t* sf, const uint32_t* amax_bits, float* g_out, RowMap map,
-                               cudaStream_t st) {
-  const int64_t mpad = ((M + 127) / 128) * 128;
-  const int64_t kch = sf_kchunks(K);
-  const int64_t total = mpad * kch * 4;
+                               uint8_t* sf, int sf_layout, const uint32_t* amax_bits,
+                               float* g_out, RowMap map, cudaStream_t st) {
+  // weights (layout 1) pad rows to the 256-row N tile, activations to 128
+  const int64_t mpad = sf_layout == 1 ? ((M + 255) / 256) * 256 : ((M + 127) / 128) * 128;
+  const int64_t nks = sfb_stages(K);  // == sf_kchunks(K) / 4
+  const int64_t total = mpad * nks * 4;
   if (total <= 0) return cudaSuccess;
   const int64_t blocks = (total + 255) / 256;
   quant_nvfp4_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(x), M, K, ldx, q, sf, kch, mpad, amax_bits, g_out, map);
+      static_cast<const __nv_bfloat16*>(x), M, K, ldx, q, sf, sf_layout, nks, mpad, amax_bits,
+      g_out, map);
   return cudaGetLastError();
 }
 

@@ -78,6 +78,9 @@ def test_create_rejects_before_any_cuda_call():
     bad = ql.make_desc("fp8", "bias", 512, 256, flags=1)
     s, h = ql.qlinear_create(bad, 0x1000, None, 0x100000, 1 << 30, check=False)
     assert s == _abi.QL_ERR_INVALID_ARG
+    bad = ql.make_desc("fp8", "bias", 512, 256, variant=3)
+    s, h = ql.qlinear_create(bad, 0x1000, None, 0x100000, 1 << 30, check=False)
+    assert s == _abi.QL_ERR_INVALID_ARG
 
 
 def test_null_handle_calls():

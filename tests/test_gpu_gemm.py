@@ -13,7 +13,8 @@ pytestmark = pytest.mark.gpu
 EPIS = ["bias", "bias_gelu", "swiglu", "bias_gated_residual", "split_bias_gelu"]
 
 
-def _run(fmt, epi, M, N, K, seed=0, x_kind="normal", bias=True, rows=None, split_col=None):
+def _run(fmt, epi, M, N, K, seed=0, x_kind="normal", bias=True, rows=None, split_col=None,
+         variant=0):
     import torch
     import precision_gemm_qlinear_b200 as ql
     if x_kind == "normal":
@@ -28,7 +29,8 @@ def _run(fmt, epi, M, N, K, seed=0, x_kind="normal", bias=True, rows=None, split
     if epi == "bias_gated_residual":
         gate = draw("normal", (Nout,), seed, "gate", mean=1.0, std=0.1)
         res = draw("normal", (M, Nout), seed, "residual")
-    lay = ql.QLinear(fmt, epi, to_dev_bf16(w), None if b is None else to_dev_bf16(b), split_col=sc)
+    lay = ql.QLinear(fmt, epi, to_dev_bf16(w), None if b is None else to_dev_bf16(b), split_col=sc,
+                     variant=variant)
     out = lay(to_dev_bf16(x), residual=None if res is None else to_dev_bf16(res),
               gate=None if gate is None else to_dev_bf16(gate))
     torch.cuda.synchronize()
@@ -41,13 +43,15 @@ def _run(fmt, epi, M, N, K, seed=0, x_kind="normal", bias=True, rows=None, split
     return got, ref["out"]
 
 
+@pytest.mark.parametrize("variant", [1, 2])
 @pytest.mark.parametrize("epi", EPIS)
 @pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
-def test_small_all_epilogues(fmt, epi):
-    # 3 M tiles with a ragged tail, 2-3 N tiles, several K stages
+def test_small_all_epilogues(fmt, epi, variant):
+    # 3 M tiles (one CTA) / 2 pair tiles with a ragged tail, 2-3 N tiles,
+    # several K stages; variant 1 = one CTA per 128-row tile, 2 = CTA pairs
     K = 384 if fmt == "fp8" else 512
-    got, ref = _run(fmt, epi, 300, 768 if epi != "swiglu" else 1024, K)
-    assert_close(got, ref, f"{fmt}/{epi}")
+    got, ref = _run(fmt, epi, 300, 768 if epi != "swiglu" else 1024, K, variant=variant)
+    assert_close(got, ref, f"{fmt}/{epi}/v{variant}")
 
 
 @pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
@@ -56,9 +60,10 @@ def test_tiny_config(fmt):
     assert_close(got, ref, f"tiny {fmt}")
 
 
-@pytest.mark.parametrize("M", [1, 5, 127, 129])
-def test_ragged_m(M):
-    got, ref = _run("fp8", "bias", M, 512, 256)
+@pytest.mark.parametrize("variant", [0, 2])
+@pytest.mark.parametrize("M", [1, 5, 127, 129, 255, 257])
+def test_ragged_m(M, variant):
+    got, ref = _run("fp8", "bias", M, 512, 256, variant=variant)
     assert_close(got, ref, f"M={M}")
 
 
@@ -75,11 +80,14 @@ def test_fp8_n_not_multiple_of_tile():
     assert_close(got, ref, "N=288")
 
 
+@pytest.mark.parametrize("variant", [1, 2])
 @pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
-def test_many_tiles_per_cta(fmt):
-    # more tiles than SMs: every CTA runs several tiles and cycles both TMEM
-    # accumulator buffers; oracle on a row sample covering every M tile
-    M, N, K = 2000, 2560, 256
+def test_many_tiles_per_cta(fmt, variant):
+    # more tiles than SMs (or CTA pairs): every CTA runs several tiles and
+    # cycles both TMEM accumulator buffers; oracle on a row sample covering
+    # every M tile
+    M, N, K = 2000, 2560 if variant == 1 else 5120, 256
     rows = sample_rows(M, 48, seed=1)
-    got, ref = _run(fmt, "split_bias_gelu", M, N, K, x_kind="t", rows=rows, split_col=1024)
-    assert_close(got, ref, f"many tiles {fmt}")
+    got, ref = _run(fmt, "split_bias_gelu", M, N, K, x_kind="t", rows=rows, split_col=1024,
+                    variant=variant)
+    assert_close(got, ref, f"many tiles {fmt} v{variant}")

@@ -61,7 +61,7 @@ def test_nvfp4_act_quant_bitexact(M, K, dist):
     assert np.float32(gg).view(np.uint32) == np.float32(rg).view(np.uint32)
     assert np.array_equal(gsf, rsf)
     assert np.array_equal(gc, rc)
-    # every padding scale byte is zero
+    # every padding scale byte (rows >= M, blocks >= K/16) is zero
     mask = np.ones(nsf, bool)
     r = np.arange(M)[:, None]
     b = np.arange(K // 16)[None, :]

@@ -3,7 +3,7 @@
 import numpy as np
 import pytest
 
-from qlutil import sf_layout_offsets, sf_unswizzle
+from qlutil import sf_layout_offsets, sf_unswizzle, sfb_word_offsets
 
 
 @pytest.mark.parametrize("rows,K", [(1, 32), (128, 256), (300, 3072), (257, 544), (16896, 3072)])
@@ -24,3 +24,14 @@ def test_sf_unswizzle_roundtrip():
         for b in range(K // 16):
             buf[((r // 128) * kch + b // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + b % 4] = logical[r, b]
     assert np.array_equal(sf_unswizzle(buf, rows, K), logical)
+
+
+
+@pytest.mark.parametrize("N,K", [(256, 32), (512, 256), (768, 3072), (256, 544)])
+def test_weight_sf_layout_words_tile_the_buffer(N, K):
+    # every (row, stage, step, replica) word has its own 4-byte slot and the
+    # slots cover the buffer exactly
+    off = sfb_word_offsets(N, K).ravel()
+    total = ((N + 255) // 256) * ((K + 255) // 256) * 4 * 4096
+    assert np.all(off % 4 == 0)
+    assert np.array_equal(np.sort(off), np.arange(0, total, 4))
