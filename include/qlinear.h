@@ -127,6 +127,33 @@ QL_API ql_status qlinear_out_features(qlinear_t h, int64_t* nout);
 QL_API ql_status qlinear_quantize_act(qlinear_t h, const void* x_bf16, int64_t M, void* codes,
                                void* scales, void* stream);
 
+/* Largest M accepted by qlinear_quantize_act_noalloc for NVFP4 layers. */
+#define QL_NOALLOC_MAX_ROWS 524288
+
+/* Activation quantization for callers that cannot allocate device memory.
+ * The pages have no counterpart of this call; it exists for callers that are
+ * not allowed to call cudaMalloc or to own a scratch buffer -- code running
+ * inside another framework's memory pool, an operator plugin that is handed
+ * only its input and output tensors, or a graph-replay path that must not
+ * touch the allocator.
+ *   Arguments and outputs are those of qlinear_quantize_act (the caller still
+ *   provides x, codes and scales, sized by qlinear_act_bytes).  FP8 layers use
+ *   the same single-pass kernel, which needs no working memory.  For NVFP4
+ *   the working memory of the tensor-amax reduction (one partial maximum per
+ *   128-row block, then the tensor maximum) is a fixed array inside the
+ *   library (QL_NOALLOC_MAX_ROWS / 128 + 64 words per device, held until the
+ *   process exits) instead of the amax word in the scales tail.
+ *   M > QL_NOALLOC_MAX_ROWS returns QL_ERR_INVALID_ARG before any launch.
+ *   The first call on a device looks up that array's device address (no
+ *   allocation); make that first call before any stream capture.
+ *   All calls on a device share the array and it keeps the last call's
+ *   contents; no entry of it needs to start at zero, because every call
+ *   writes the entries it reads.  Calls whose kernels overlap on the GPU
+ *   (other streams, other host threads) race on the array: order them.
+ *   No device memory is allocated or freed, no host sync. */
+QL_API ql_status qlinear_quantize_act_noalloc(qlinear_t h, const void* x_bf16, int64_t M,
+                                              void* codes, void* scales, void* stream);
+
 /* GEMM + fused epilogue (no host sync, no allocation).
  *   codes, scales : as written by qlinear_quantize_act for the same M.
  *   residual      : device [M, Nout] bf16 for QL_EPI_BIAS_GATED_RESIDUAL, else NULL.

@@ -18,8 +18,9 @@ EPILOGUES = {"bias": 0, "bias_gelu": 1, "swiglu": 2, "bias_gated_residual": 3,
 
 # every entry point declared in include/qlinear.h
 EXPORTS = ("qlinear_weight_bytes", "qlinear_create", "qlinear_act_bytes", "qlinear_out_features",
-           "qlinear_quantize_act", "qlinear_forward", "qlinear_export_weights", "qlinear_check",
-           "qlinear_destroy", "qlinear_status_string", "qlinear_abi_version")
+           "qlinear_quantize_act", "qlinear_quantize_act_noalloc", "qlinear_forward",
+           "qlinear_export_weights", "qlinear_check", "qlinear_destroy", "qlinear_status_string",
+           "qlinear_abi_version")
 
 
 class ql_desc(ctypes.Structure):
@@ -54,6 +55,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.qlinear_act_bytes.argtypes = [P, i64, ctypes.POINTER(sz), ctypes.POINTER(sz)]
     L.qlinear_out_features.argtypes = [P, ctypes.POINTER(i64)]
     L.qlinear_quantize_act.argtypes = [P, P, i64, P, P, P]
+    L.qlinear_quantize_act_noalloc.argtypes = [P, P, i64, P, P, P]
     L.qlinear_forward.argtypes = [P, P, P, i64, P, P, P, P]
     L.qlinear_export_weights.argtypes = [P, P, P, ctypes.POINTER(ctypes.c_float), P]
     L.qlinear_check.argtypes = [P, P]
@@ -126,6 +128,17 @@ def qlinear_quantize_act(h, x_ptr, M, codes_ptr, scales_ptr, stream=0, check=Tru
     s = load().qlinear_quantize_act(h, x_ptr, M, codes_ptr, scales_ptr, stream)
     if check:
         _ck("qlinear_quantize_act", s)
+    return s
+
+
+QL_NOALLOC_MAX_ROWS = 524288
+
+
+def qlinear_quantize_act_noalloc(h, x_ptr, M, codes_ptr, scales_ptr, stream=0, check=True):
+    """Allocation-free activation quantization (working memory inside the library)."""
+    s = load().qlinear_quantize_act_noalloc(h, x_ptr, M, codes_ptr, scales_ptr, stream)
+    if check:
+        _ck("qlinear_quantize_act_noalloc", s)
     return s
 
 

@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libqlinear_b200.so")
-SOURCES = ["quant.cu", "gemm.cu", "qlinear_api.cu"]
+SOURCES = ["quant.cu", "gemm.cu", "noalloc.cu", "qlinear_api.cu"]
 HEADERS = ["ptx.cuh", "internal.h", os.path.join("..", "..", "include", "qlinear.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

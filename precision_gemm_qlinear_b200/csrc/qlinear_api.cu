@@ -17,6 +17,11 @@
 
 using namespace qlb;
 
+namespace qlb {
+ql_status quantize_act_noalloc(int fmt, int64_t K, int num_sms, const void* x, int64_t M,
+                               void* codes, void* scales, cudaStream_t st);
+}
+
 struct qlinear_s {
   ql_desc d;
   int64_t N, K, Nout;
@@ -302,6 +307,17 @@ ql_status qlinear_quantize_act(qlinear_t h, const void* x_bf16, int64_t M, void*
   }
   if (e != cudaSuccess) cudaGetLastError();
   return from_cuda(e);
+}
+
+ql_status qlinear_quantize_act_noalloc(qlinear_t h, const void* x_bf16, int64_t M, void* codes,
+                                       void* scales, void* stream) {
+  if (!h || M < 0 || M > 0x7FFFFFFF) return QL_ERR_INVALID_ARG;
+  if (h->d.fmt == QL_NVFP4 && M > QL_NOALLOC_MAX_ROWS) return QL_ERR_INVALID_ARG;
+  if (M == 0) return QL_OK;
+  if (!x_bf16 || !codes || !scales) return QL_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scales)) return QL_ERR_ALIGNMENT;
+  return qlb::quantize_act_noalloc(h->d.fmt, h->K, h->num_sms, x_bf16, M, codes, scales,
+                                   static_cast<cudaStream_t>(stream));
 }
 
 ql_status qlinear_forward(qlinear_t h, const void* codes, const void* scales, int64_t M,
