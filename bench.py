@@ -148,6 +148,30 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.samples)}
 
 
+# ------------------------------------------------------- multi-rank helpers
+
+def rank_seed(rank: int) -> int:
+    """Weak scaling over tokens: every rank quantizes and multiplies its own
+    tokens (seed = rank), against the same weights (seed 0)."""
+    return int(rank)
+
+
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """Max of a per-rank device time over all ranks (the job's time)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_tflops(flops_per_step: float, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: the FLOPs of every rank over the slowest rank's time."""
+    return flops_per_step * world * steps / (max_ms / 1e3) / 1e12
+
+
 # --------------------------------------------------------------------- ours
 
 def to_dev(a, dev):
@@ -167,7 +191,7 @@ class Model:
         for s in range(nsets):
             layers = []
             for li, layer in enumerate(wl.layers):
-                inp = make_inputs(layer, seed=seed * 1000 + s, layer_index=li)
+                inp = make_inputs(layer, seed=seed * 1000 + s, layer_index=li, w_seed=s)
                 if s == 0 and li == 0:
                     host0 = inp
                 lay = ql.QLinear(layer.fmt, layer.epi, to_dev(inp["w"], dev),
@@ -266,7 +290,7 @@ def main_ours(args):
         per_set += layer.M * layer.K * 2 + layer.N * kb + layer.M * (
             layer.N // 2 if layer.epi == "swiglu" else layer.N) * 2
     nsets = args.sets or max(2, int(np.ceil(2 * L2_BYTES / per_set)) + 1)
-    model = Model(wl, dev, seed=rank, nsets=nsets)
+    model = Model(wl, dev, seed=rank_seed(rank), nsets=nsets)
     stream = torch.cuda.Stream(device=dev)
     flops_step = float(wl.flops)
 
@@ -308,12 +332,9 @@ def main_ours(args):
             if st != 0:
                 raise RuntimeError(f"device error during timing: status {st}")
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = max_ms / args.steps
-    value = flops_step * world * args.steps / (max_ms / 1e3) / 1e12
+    value = weak_scaling_tflops(flops_step, world, args.steps, max_ms)
 
     # dominant kernel: the GEMM with the largest time share
     j = int(np.argmax(gemm_ms))
@@ -402,13 +423,8 @@ def run_e2e(model, stream, dev, args, world, flops_step):
             one()
         e1.record(stream)
         stream.synchronize()
-    ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
-    return {"value": round(flops_step * world * steps / (ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    return {"value": round(weak_scaling_tflops(flops_step, world, steps, ms), 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(x_host.numel() * 2),
             "d2h_bytes_per_step": int(out_host.numel() * 2), "steps": steps}
 

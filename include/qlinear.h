@@ -178,6 +178,15 @@ QL_API ql_status qlinear_check(qlinear_t h, void* stream);
 /* Release the host handle (the caller frees weight_ws afterwards). */
 QL_API ql_status qlinear_destroy(qlinear_t h);
 
+/* Test hook for the device-side watchdog (no counterpart on the pages).
+ * mode 1: in every later qlinear_forward on this handle, the first CTA's TMA
+ * producer leaves its first pipeline stage unfilled, so the MMA thread's
+ * bounded wait (about one second) expires; the kernel records the expiry,
+ * drains what it issued and exits, and qlinear_check returns QL_ERR_TIMEOUT.
+ * The output of such a call is incomplete.  mode 0 restores normal operation.
+ * Host only, no CUDA call. */
+QL_API ql_status qlinear_debug_set_fault(qlinear_t h, int32_t mode);
+
 /* Static description of a status code. */
 QL_API const char* qlinear_status_string(ql_status s);
 

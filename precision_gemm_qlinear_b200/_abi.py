@@ -19,8 +19,8 @@ EPILOGUES = {"bias": 0, "bias_gelu": 1, "swiglu": 2, "bias_gated_residual": 3,
 # every entry point declared in include/qlinear.h
 EXPORTS = ("qlinear_weight_bytes", "qlinear_create", "qlinear_act_bytes", "qlinear_out_features",
            "qlinear_quantize_act", "qlinear_quantize_act_noalloc", "qlinear_forward",
-           "qlinear_export_weights", "qlinear_check", "qlinear_destroy", "qlinear_status_string",
-           "qlinear_abi_version")
+           "qlinear_export_weights", "qlinear_check", "qlinear_debug_set_fault", "qlinear_destroy",
+           "qlinear_status_string", "qlinear_abi_version")
 
 
 class ql_desc(ctypes.Structure):
@@ -59,6 +59,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.qlinear_forward.argtypes = [P, P, P, i64, P, P, P, P]
     L.qlinear_export_weights.argtypes = [P, P, P, ctypes.POINTER(ctypes.c_float), P]
     L.qlinear_check.argtypes = [P, P]
+    L.qlinear_debug_set_fault.argtypes = [P, ctypes.c_int32]
     L.qlinear_destroy.argtypes = [P]
     L.qlinear_status_string.argtypes = [st]
     L.qlinear_status_string.restype = ctypes.c_char_p
@@ -163,3 +164,7 @@ def qlinear_check(h, stream=0):
 
 def qlinear_destroy(h):
     _ck("qlinear_destroy", load().qlinear_destroy(h))
+
+
+def qlinear_debug_set_fault(h, mode):
+    _ck("qlinear_debug_set_fault", load().qlinear_debug_set_fault(h, mode))

@@ -37,6 +37,7 @@ struct qlinear_s {
   uint32_t* wamax;   // NVFP4 amax word used while quantizing W
   __nv_bfloat16* bias;
   RowMap map;
+  int32_t fault_mode;  // test hook, see qlinear_debug_set_fault
   CUtensorMap tmB1;    // weight codes, box 128 B x 256 rows (one CTA per tile)
   CUtensorMap tmB2;    // weight codes, box 128 B x 128 rows (CTA pair per tile)
   CUtensorMap tmSFB;   // NVFP4: weight SF atoms as 2048-byte rows (CTA pair)
@@ -370,7 +371,7 @@ ql_status qlinear_forward(qlinear_t h, const void* codes, const void* scales, in
   p.group_m = 8;
   p.sf_kchunks_a = static_cast<int32_t>(sf_kchunks(h->K));
   p.sfb_nstages = static_cast<int32_t>(sfb_stages(h->K));
-  p.fault_mode = 0;
+  p.fault_mode = h->fault_mode;
   cudaError_t e =
       launch_gemm(h->d.fmt, h->d.epi, cg, p, h->num_sms, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
@@ -441,6 +442,12 @@ ql_status qlinear_check(qlinear_t h, void* stream) {
     cudaMemcpy(h->err, &zero, 4, cudaMemcpyHostToDevice);
     return QL_ERR_TIMEOUT;
   }
+  return QL_OK;
+}
+
+ql_status qlinear_debug_set_fault(qlinear_t h, int32_t mode) {
+  if (!h || mode < 0 || mode > 1) return QL_ERR_INVALID_ARG;
+  h->fault_mode = mode;
   return QL_OK;
 }
 

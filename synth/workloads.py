@@ -76,23 +76,27 @@ WORKLOADS = {
 }
 
 
-def make_inputs(layer: Layer, seed: int = 0, layer_index: int = 0, M: int = None):
+def make_inputs(layer: Layer, seed: int = 0, layer_index: int = 0, M: int = None,
+                w_seed: int = None):
     """Draw the host-side bf16 tensors of one layer (uint16 bit patterns).
 
     Returns dict with x [M,K] (absent when chained), w [N,K], bias [N] or None,
-    gate [Nout] and residual [M,Nout] for the gated-residual epilogue.
+    gate [Nout] and residual [M,Nout] for the gated-residual epilogue.  The
+    per-token tensors (x, residual) come from `seed`; the layer's parameters
+    (w, bias, gate) from `w_seed` (default: `seed`).
     """
     M = layer.M if M is None else M
+    ws = seed if w_seed is None else w_seed
     sfx = "" if layer_index == 0 else "2"
     out = {}
     if not layer.chained:
         d = dict(layer.x_dist)
         kind = d.pop("kind")
         out["x"] = draw(kind, (M, layer.K), seed, "x" + sfx, **d)
-    out["w"] = draw("normal", (layer.N, layer.K), seed, "w" + sfx, std=layer.w_std)
+    out["w"] = draw("normal", (layer.N, layer.K), ws, "w" + sfx, std=layer.w_std)
     out["bias"] = (None if layer.bias_std is None else
-                   draw("normal", (layer.N,), seed, "bias" + sfx, std=layer.bias_std))
+                   draw("normal", (layer.N,), ws, "bias" + sfx, std=layer.bias_std))
     if layer.epi == "bias_gated_residual":
-        out["gate"] = draw("normal", (layer.Nout,), seed, "gate", mean=1.0, std=0.1)
+        out["gate"] = draw("normal", (layer.Nout,), ws, "gate", mean=1.0, std=0.1)
         out["residual"] = draw("normal", (M, layer.Nout), seed, "residual", std=1.0)
     return out
