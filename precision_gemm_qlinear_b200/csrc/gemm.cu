@@ -43,7 +43,6 @@ namespace qlb {
 namespace {
 
 constexpr int BM = 128;                // rows of the tile per CTA
-constexpr int BN = 256;                // columns of the tile (MMA N)
 constexpr int BK_BYTES = 128;          // K bytes per pipeline stage
 constexpr int A_BYTES = BM * BK_BYTES;  // 16 KB
 constexpr int NUM_EPI_WARPS = 8;
@@ -58,37 +57,46 @@ constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // 1 s
 //  kind::mxf4nvf4: [4,6) B scale id, [7,10) A fmt (1 = E2M1), [10,13) B fmt,
 //                 [17,23) N>>3, [23] scale type (0 = UE4M3), [24,29) M>>4,
 //                 [29,31) A scale id, [31] K size (0 = 64).
-template <int CG>
+template <int CG, int BN>
 constexpr uint32_t idesc_f8() {
   return (1u << 4) | (0u << 7) | (0u << 10) | ((BN >> 3) << 17) | (((BM * CG) >> 4) << 24);
 }
-template <int CG>
+template <int CG, int BN>
 constexpr uint32_t idesc_f4() {
   return (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | (((BM * CG) >> 4) << 24);
 }
 
-template <int FMT, int CG>
+template <int FMT, int CG, int EPI>
 struct Cfg {
   static constexpr bool NV = (FMT == 1);
   static constexpr bool PAIR = (CG == 2);
+  // Tile N: 256, except NVFP4 without SwiGLU, where 224 lets two fp32
+  // accumulators (2 x 224 TMEM columns) and the 48 scale-factor columns fit
+  // in the 512 columns side by side.
+  static constexpr int BN = (NV && EPI != EPI_SWIGLU) ? 224 : 256;
   static constexpr int B_BYTES = (BN / CG) * BK_BYTES;  // this CTA's rows of B
   static constexpr int SFA_BYTES = NV ? 2048 : 0;       // 4 atoms (one per MMA K step)
   static constexpr int SFB_BYTES = NV ? 16384 : 0;      // 4 replicated 4 KB chunks (all 256 B rows)
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int STAGES = NV ? (PAIR ? 4 : 3) : (PAIR ? 6 : 4);
-  static constexpr int NBUF = NV ? 1 : 2;  // staging buffers per epilogue warp
+  // staging buffers per epilogue warp: two unless that breaks the budget
+  static constexpr int NBUF =
+      (STAGES * STAGE_BYTES + NUM_EPI_WARPS * 2 * STAGING_BYTES + 256 + 1024 <= 232448) ? 2 : 1;
   static constexpr int STAGING_OFF = STAGES * STAGE_BYTES;
   static constexpr int BAR_OFF = STAGING_OFF + NUM_EPI_WARPS * NBUF * STAGING_BYTES;
   static_assert(BAR_OFF + 256 + 1024 <= 232448, "shared memory budget");
   static constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
-  // TMEM columns: FP8 -> two disjoint 256-column accumulators.
-  // NVFP4 -> accumulators at 0 and 192 (overlapping in [192,256)); the scale
-  // factors of the current stage live in [448, 496): A in 4 x 4 columns, B in
-  // 4 x 8 columns (one group per 64-element MMA step).
-  static constexpr uint32_t ACC1 = NV ? 192 : 256;
+  // TMEM columns: FP8 -> two disjoint 256-column accumulators.  NVFP4 ->
+  // the scale factors of the current stage live in [448, 496) (A in 4 x 4
+  // columns, B in 4 x 8, one group per 64-element MMA step); with N = 224 the
+  // accumulators are [0,224) and [224,448); with N = 256 (SwiGLU) they are
+  // [0,256) and [192,448), overlapping in [192,256), and the epilogue reads
+  // the shared columns first and releases them early.
+  static constexpr bool OVL = NV && BN == 256;
+  static constexpr uint32_t ACC1 = OVL ? 192 : BN;
   static constexpr uint32_t SFA_COL = 448;
   static constexpr uint32_t SFB_COL = 464;
-  static constexpr bool OVL = NV;
+  static_assert(!NV || ACC1 + BN <= SFA_COL, "TMEM budget");
   static constexpr uint32_t EPI_ARRIVALS = NUM_EPI_WARPS * CG;  // per tile, at the leader
 };
 
@@ -134,13 +142,38 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, SmemBar
   }
 }
 
-__device__ __forceinline__ float gelu_tanh_f(float v) {
-  // 0.5 v (1 + tanh(u)) = v * sigmoid(2u), u = sqrt(2/pi) (v + 0.044715 v^3)
-  const float u2 = 1.5957691216057308f * fmaf(0.044715f * v, v * v, v);
-  return __fdividef(v, 1.0f + __expf(-u2));
+// The GELU / SiLU epilogues are bound by the special-function unit, so each
+// element uses exactly one SFU operation (the base-2 exponential) and takes
+// the reciprocal on the FMA pipe: Newton-Raphson r <- r (2 - d r) from the
+// classic exponent-bit initial guess, three steps (relative error < 2e-7 for
+// d >= 1).
+__device__ __forceinline__ float ex2_sfu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+__device__ __forceinline__ float rcp_newton(float d) {  // d >= 1, finite
+  float r = __int_as_float(0x7EF311C7 - __float_as_int(d));
+  r = r * fmaf(-d, r, 2.0f);
+  r = r * fmaf(-d, r, 2.0f);
+  r = r * fmaf(-d, r, 2.0f);
+  return r;
+}
+
+__device__ __forceinline__ float gelu_tanh_f(float v) {
+  // 0.5 v (1 + tanh(u)) = v / (1 + e^{-2u}), u = sqrt(2/pi) v (1 + 0.044715 v^2);
+  // e^{-2u} = 2^{-2 u log2(e)}; the exponent is clamped so 1 + e stays finite
+  const float t = fmaf(0.044715f * v, v, 1.0f);
+  const float x = fminf(-2.3022081983953454f * v * t, 126.0f);  // -2 sqrt(2/pi) log2(e)
+  return v * rcp_newton(1.0f + ex2_sfu(x));
+}
+
+__device__ __forceinline__ float silu_f(float g) {
+  // g / (1 + e^{-g}),  e^{-g} = 2^{-g log2(e)}
+  const float x = fminf(-1.4426950408889634f * g, 126.0f);
+  return g * rcp_newton(1.0f + ex2_sfu(x));
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -163,6 +196,19 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* p, float (&o)[
   }
 }
 
+// 32 bf16 kept packed (16 registers); element i is bf16x32_at(v, i).
+__device__ __forceinline__ void load_bf16x32_packed(const __nv_bfloat16* p, uint4 (&v)[4]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __ldg(q + i);
+}
+__device__ __forceinline__ float bf16x32_at(const uint4 (&v)[4], int i) {
+  const uint4& w = v[i >> 3];
+  const int k = (i >> 1) & 3;
+  const uint32_t word = k == 0 ? w.x : (k == 1 ? w.y : (k == 2 ? w.z : w.w));
+  return (i & 1) ? bf16hi(word) : bf16lo(word);
+}
+
 __device__ __forceinline__ void load_f32x32(const float* p, float (&o)[32]) {
   const float4* q = reinterpret_cast<const float4*>(p);
 #pragma unroll
@@ -177,7 +223,8 @@ __device__ __forceinline__ void load_f32x32(const float* p, float (&o)[32]) {
 
 template <int FMT, int EPI, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_constant__ GemmParams p) {
-  using C = Cfg<FMT, CG>;
+  using C = Cfg<FMT, CG, EPI>;
+  constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -352,16 +399,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
             const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
             if constexpr (C::NV) {
               if constexpr (C::PAIR)
-                mma_mxf4nvf4_pair(d_tmem, ad, bd, idesc_f4<CG>(), tmem + C::SFA_COL + 4 * j,
+                mma_mxf4nvf4_pair(d_tmem, ad, bd, idesc_f4<CG, BN>(), tmem + C::SFA_COL + 4 * j,
                                   tmem + C::SFB_COL + 8 * j, acc);
               else
-                mma_mxf4nvf4(d_tmem, ad, bd, idesc_f4<CG>(), tmem + C::SFA_COL + 4 * j,
+                mma_mxf4nvf4(d_tmem, ad, bd, idesc_f4<CG, BN>(), tmem + C::SFA_COL + 4 * j,
                              tmem + C::SFB_COL + 8 * j, acc);
             } else {
               if constexpr (C::PAIR)
-                mma_f8f6f4_pair(d_tmem, ad, bd, idesc_f8<CG>(), acc);
+                mma_f8f6f4_pair(d_tmem, ad, bd, idesc_f8<CG, BN>(), acc);
               else
-                mma_f8f6f4(d_tmem, ad, bd, idesc_f8<CG>(), acc);
+                mma_f8f6f4(d_tmem, ad, bd, idesc_f8<CG, BN>(), acc);
             }
           }
           any = true;
@@ -396,9 +443,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
     // --------------------------------------------------------- epilogue
     const int ew = warp - 2;           // 0..7
     const int sp = warp & 3;           // TMEM sub-partition: rows [32 sp, 32 sp + 32) of the CTA tile
-    const int half = ew >> 2;          // which half of the tile's columns this warp owns
+    const int half = ew >> 2;          // the two warps of a sub-partition take alternate chunks
     uint8_t* staging = smem + C::STAGING_OFF + ew * C::NBUF * STAGING_BYTES;
-    constexpr int NCH = (EPI == EPI_SWIGLU) ? 2 : 4;  // 32-column output chunks per warp per tile
+    // 32-column output chunks per tile, and this warp's share of them
+    constexpr int NCHT = (EPI == EPI_SWIGLU) ? BN / 64 : BN / 32;
+    const int nch = (NCHT - half + 1) >> 1;
     const uint32_t ovl_l0 = mapa_shared(smem_u32(&sb->ovl_free), 0);
     int local = 0;
     uint32_t nstore = 0;
@@ -409,14 +458,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
       const uint32_t use = static_cast<uint32_t>(local >> 1);
       if (!wait_bar(&sb->acc_full[buf], use & 1, sb, p.err, ERR_WAIT_EPI)) break;
       tc_fence_after();
-      // NVFP4: the accumulator columns shared by the two TMEM buffers belong to
-      // half 1 of buffer 0 and half 0 of buffer 1; those warps read them first
-      // and then release the overlap so the next tile's MMA can start.
-      const bool ovl_owner = C::OVL && (half == (buf == 0 ? 1 : 0));
-      if (C::OVL && !ovl_owner) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(ovl_l0);
-      }
       const int row0 = mb * (BM * CG) + static_cast<int>(rank) * BM + sp * 32;  // first row of this warp
       const int m = row0 + lane;
       const bool row_ok = m < p.M;
@@ -427,93 +468,121 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
       else
         rs = row_ok ? __ldg(p.sa + m) : 0.f;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(sp * 32) << 16) + (buf ? C::ACC1 : 0u);
-      for (int ci = 0; ci < NCH; ++ci) {
-        const int lc = (ovl_owner && buf == 0) ? (ci + 2) % NCH : ci;
-        const int c = half * NCH + lc;  // chunk index within the tile (output chunks for SwiGLU)
-        uint32_t ra[32];
-        tmem_ld_32x32b_x32(tbase + 32 * c, ra);
-        uint32_t rb[32];
-        if constexpr (EPI == EPI_SWIGLU) tmem_ld_32x32b_x32(tbase + 128 + 32 * c, rb);
+      // chunk processed at step ci.  SwiGLU with overlapping buffers: the
+      // shared columns are the up half of output chunks 2, 3 in buffer 0 and
+      // the gate half of chunks 0, 1 in buffer 1; every warp holds exactly one
+      // of them and reads it first.
+      auto chunk_of = [&](int ci) {
+        const int k = (C::OVL && buf == 0) ? (nch - 1 - ci) : ci;
+        return half + 2 * k;
+      };
+      constexpr int NCHW = (NCHT + 1) / 2;  // most chunks a warp can have
+      uint32_t acc[2][32];                   // double-buffered accumulator chunk
+      uint32_t accu[32];                     // SwiGLU: the up half
+      tmem_ld_32x32b_x32(tbase + 32 * chunk_of(0), acc[0]);
+      if constexpr (EPI == EPI_SWIGLU) tmem_ld_32x32b_x32(tbase + 128 + 32 * chunk_of(0), accu);
+#pragma unroll
+      for (int ci = 0; ci < NCHW; ++ci) {
+        if (ci >= nch) break;
+        const int c = chunk_of(ci);
+        const int ncol = nb * BN + 32 * c;                                     // GEMM column of acc[..][0]
+        const int ocol = (EPI == EPI_SWIGLU) ? nb * (BN / 2) + 32 * c : ncol;  // output column
+        // SwiGLU (N = 256): gate columns ncol.., up columns ncol + 128..
+        const bool live = ncol < p.N;  // past the last column (N % 32 == 0); warp-uniform
+        // per-column and per-row operands: issued before the TMEM wait so the
+        // two latencies overlap
+        uint4 bias_a[4], bias_b[4], gate_a[4], res_a[4];
+        float sw_a[32], sw_b[32];
+        if (live) {
+          load_bf16x32_packed(p.bias + ncol, bias_a);
+          if constexpr (!C::NV) load_f32x32(p.sw + ncol, sw_a);
+          if constexpr (EPI == EPI_SWIGLU) {
+            load_bf16x32_packed(p.bias + ncol + 128, bias_b);
+            if constexpr (!C::NV) load_f32x32(p.sw + ncol + 128, sw_b);
+          }
+          if constexpr (EPI == EPI_GATED_RES) {
+            load_bf16x32_packed(p.gate + ocol, gate_a);
+            if (row_ok) {
+              load_bf16x32_packed(p.residual + static_cast<int64_t>(m) * p.Nout + ocol, res_a);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) res_a[i] = make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
+        }
         tmem_wait_ld();
-        if (ovl_owner && ci == 1) {
+        // the next chunk's accumulators stream in while this one is computed
+        if constexpr (EPI != EPI_SWIGLU) {
+          if (ci + 1 < nch) tmem_ld_32x32b_x32(tbase + 32 * chunk_of(ci + 1), acc[(ci + 1) & 1]);
+        }
+        if (C::OVL && ci == 0) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(ovl_l0);
         }
-        if (ci == NCH - 1) {
+        if (ci == nch - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sb->acc_empty[buf]), 0));
         }
-        // ---- epilogue math on 32 columns of this thread's row
-        const int ncol = nb * BN + 32 * c;                                     // GEMM column of ra[0]
-        const int ocol = (EPI == EPI_SWIGLU) ? nb * (BN / 2) + 32 * c : ncol;  // output column
-        if (ncol >= p.N) continue;  // past the last column (N % 32 == 0); warp-uniform
+        const uint32_t* ra = acc[(EPI == EPI_SWIGLU) ? 0 : (ci & 1)];
         uint32_t packed[16];
-        float bias_a[32];
-        load_bf16x32(p.bias + ncol, bias_a);
-        if constexpr (EPI == EPI_SWIGLU) {
-          float bias_b[32];
-          load_bf16x32(p.bias + ncol + 128, bias_b);
-          float sw_a[32], sw_b[32];
-          if constexpr (!C::NV) {
-            load_f32x32(p.sw + ncol, sw_a);
-            load_f32x32(p.sw + ncol + 128, sw_b);
-          }
+        if (live) {
+          if constexpr (EPI == EPI_SWIGLU) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float o[2];
+            for (int i = 0; i < 32; i += 2) {
+              float o[2];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              float sa_, sb_;
-              if constexpr (C::NV) {
-                sa_ = rs;
-                sb_ = rs;
-              } else {
-                sa_ = rs * sw_a[i + h];
-                sb_ = rs * sw_b[i + h];
+              for (int h = 0; h < 2; ++h) {
+                float sa_, sb_;
+                if constexpr (C::NV) {
+                  sa_ = rs;
+                  sb_ = rs;
+                } else {
+                  sa_ = rs * sw_a[i + h];
+                  sb_ = rs * sw_b[i + h];
+                }
+                const float g = fmaf(__uint_as_float(ra[i + h]), sa_, bf16x32_at(bias_a, i + h));
+                const float u = fmaf(__uint_as_float(accu[i + h]), sb_, bf16x32_at(bias_b, i + h));
+                o[h] = silu_f(g) * u;
               }
-              const float g = fmaf(__uint_as_float(ra[i + h]), sa_, bias_a[i + h]);
-              const float u = fmaf(__uint_as_float(rb[i + h]), sb_, bias_b[i + h]);
-              o[h] = silu_f(g) * u;
+              packed[i >> 1] = pack_bf16x2(o[0], o[1]);
             }
-            packed[i >> 1] = pack_bf16x2(o[0], o[1]);
-          }
-        } else {
-          float sw_a[32];
-          if constexpr (!C::NV) load_f32x32(p.sw + ncol, sw_a);
-          float gate_a[32], res_a[32];
-          if constexpr (EPI == EPI_GATED_RES) {
-            load_bf16x32(p.gate + ocol, gate_a);
-            if (row_ok) {
-              load_bf16x32(p.residual + static_cast<int64_t>(m) * p.Nout + ocol, res_a);
-            } else {
+          } else {
+            const bool gelu_chunk =
+                (EPI == EPI_BIAS_GELU) || (EPI == EPI_SPLIT && ncol >= p.split_col);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) res_a[i] = 0.f;
-            }
-          }
-          const bool gelu_chunk =
-              (EPI == EPI_BIAS_GELU) || (EPI == EPI_SPLIT && ncol >= p.split_col);
+            for (int i = 0; i < 32; i += 2) {
+              float o[2];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float o[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              float s_;
-              if constexpr (C::NV)
-                s_ = rs;
-              else
-                s_ = rs * sw_a[i + h];
-              float v = fmaf(__uint_as_float(ra[i + h]), s_, bias_a[i + h]);
-              if constexpr (EPI == EPI_GATED_RES) v = fmaf(gate_a[i + h], v, res_a[i + h]);
-              if constexpr (EPI == EPI_BIAS_GELU || EPI == EPI_SPLIT) {
-                if (gelu_chunk) v = gelu_tanh_f(v);
+              for (int h = 0; h < 2; ++h) {
+                float s_;
+                if constexpr (C::NV)
+                  s_ = rs;
+                else
+                  s_ = rs * sw_a[i + h];
+                float v = fmaf(__uint_as_float(ra[i + h]), s_, bf16x32_at(bias_a, i + h));
+                if constexpr (EPI == EPI_GATED_RES)
+                  v = fmaf(bf16x32_at(gate_a, i + h), v, bf16x32_at(res_a, i + h));
+                if constexpr (EPI == EPI_BIAS_GELU || EPI == EPI_SPLIT) {
+                  if (gelu_chunk) v = gelu_tanh_f(v);
+                }
+                o[h] = v;
               }
-              o[h] = v;
+              packed[i >> 1] = pack_bf16x2(o[0], o[1]);
             }
-            packed[i >> 1] = pack_bf16x2(o[0], o[1]);
           }
         }
+        if constexpr (EPI == EPI_SWIGLU) {
+          // SwiGLU holds two halves per chunk; the next pair is loaded here,
+          // into the same registers
+          if (ci + 1 < nch) {
+            const int cn = chunk_of(ci + 1);
+            tmem_ld_32x32b_x32(tbase + 32 * cn, acc[0]);
+            tmem_ld_32x32b_x32(tbase + 128 + 32 * cn, accu);
+          }
+        }
+        if (!live) continue;
         // ---- stage through swizzled shared memory, then one TMA store per warp
         uint8_t* sbuf = staging + (nstore % C::NBUF) * STAGING_BYTES;
         if (lane == 0) bulk_wait_group_read<C::NBUF - 1>();
@@ -553,7 +622,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
 
 template <int FMT, int EPI, int CG>
 cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t st) {
-  using C = Cfg<FMT, CG>;
+  using C = Cfg<FMT, CG, EPI>;
   static bool attr_set = false;
   auto kern = qgemm_kernel<FMT, EPI, CG>;
   if (!attr_set) {
@@ -583,9 +652,9 @@ cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t st) {
 
 }  // namespace
 
-int gemm_smem_bytes(int fmt, int cg) {
-  if (fmt == 0) return cg == 2 ? Cfg<0, 2>::SMEM_BYTES : Cfg<0, 1>::SMEM_BYTES;
-  return cg == 2 ? Cfg<1, 2>::SMEM_BYTES : Cfg<1, 1>::SMEM_BYTES;
+int gemm_tile_n(int fmt, int epi) {
+  if (fmt == 0) return Cfg<0, 2, EPI_BIAS>::BN;
+  return epi == EPI_SWIGLU ? Cfg<1, 2, EPI_SWIGLU>::BN : Cfg<1, 2, EPI_BIAS>::BN;
 }
 
 cudaError_t launch_gemm(int fmt, int epi, int cg, const GemmParams& p, int num_sms,

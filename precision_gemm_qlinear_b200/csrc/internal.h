@@ -39,24 +39,26 @@ __host__ __device__ __forceinline__ int64_t sf_bytes(int64_t rows, int64_t K) {
 }
 
 // Scale-factor layout of the weight (B) operand, fed to TMEM by one
-// tcgen05.cp.128x256b per 64-element MMA step: for every 256-row N tile, every
-// stage of 256 K-elements and every MMA step j (0..3) there is a 4096-byte
-// chunk of 128 rows x 32 bytes.  Row (TMEM lane) l = 32 q + r0 holds, in word
-// w (0..7), the 4 scales of weight row 256 nb + 32 w + r0 for that step --
-// the same for every q (the replication across the four TMEM sub-partitions
-// that the MMA reads).  Chunks are ordered [nb][stage][j]; the 32-byte rows
-// are stored in the unswizzled K-major core-matrix order the copy expects:
-// 8-row groups 256 bytes apart, the two 16-byte halves of a row 128 bytes
-// apart, rows of a group 16 bytes apart.
+// tcgen05.cp.128x256b per 64-element MMA step: for every N tile of `bn` rows
+// (256, or 224), every stage of 256 K-elements and every MMA step j (0..3)
+// there is a 4096-byte chunk of 128 rows x 32 bytes.  Row (TMEM lane)
+// l = 32 q + r0 holds, in word w (0..7), the 4 scales of weight row
+// bn * tile + 32 w + r0 for that step -- the same for every q (the
+// replication across the four TMEM sub-partitions that the MMA reads).
+// Chunks are ordered [tile][stage][j]; the 32-byte rows are stored in the
+// unswizzled K-major core-matrix order the copy expects: 8-row groups 256
+// bytes apart, the two 16-byte halves of a row 128 bytes apart, rows of a
+// group 16 bytes apart.  Words past the tile (bn = 224: word 7) are zero.
 __host__ __device__ __forceinline__ int64_t sfb_stages(int64_t K) { return (K + 255) / 256; }
-__host__ __device__ __forceinline__ int64_t sfb_bytes(int64_t rows, int64_t K) {
-  return ((rows + 255) / 256) * sfb_stages(K) * 4 * 4096;
+__host__ __device__ __forceinline__ int64_t sfb_bytes(int64_t rows, int64_t K, int64_t bn) {
+  return ((rows + bn - 1) / bn) * sfb_stages(K) * 4 * 4096;
 }
 // byte offset of the scale word of weight row n, stage ks, step j, replica q
 __host__ __device__ __forceinline__ int64_t sfb_word_offset(int64_t n, int64_t ks, int64_t j,
-                                                            int64_t q, int64_t nks) {
-  const int64_t l = q * 32 + (n & 31), w = (n & 255) >> 5;
-  return (((n >> 8) * nks + ks) * 4 + j) * 4096 + (l >> 3) * 256 + (w >> 2) * 128 + (l & 7) * 16 +
+                                                            int64_t q, int64_t nks, int64_t bn) {
+  const int64_t tile = n / bn, loc = n - tile * bn;
+  const int64_t l = q * 32 + (loc & 31), w = loc >> 5;
+  return ((tile * nks + ks) * 4 + j) * 4096 + (l >> 3) * 256 + (w >> 2) * 128 + (l & 7) * 16 +
          (w & 3) * 4;
 }
 
@@ -67,9 +69,9 @@ cudaError_t launch_quant_fp8_rows(const void* x, int64_t M, int64_t K, int64_t l
 cudaError_t launch_tensor_amax(const void* x, int64_t n_elems, uint32_t* amax_bits, int num_sms,
                                cudaStream_t st);
 // sf_layout: 0 = activation (A operand) atoms [sf_offset], 1 = weight (B
-// operand) replicated chunks [sfb_word_offset].
+// operand) replicated chunks [sfb_word_offset] for N tiles of `bn` rows.
 cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
-                               uint8_t* sf, int sf_layout, const uint32_t* amax_bits,
+                               uint8_t* sf, int sf_layout, int64_t bn, const uint32_t* amax_bits,
                                float* g_out, RowMap map, cudaStream_t st);
 cudaError_t launch_permute_bias(const void* src, void* dst, int64_t N, RowMap map,
                                 cudaStream_t st);
@@ -105,7 +107,8 @@ struct alignas(64) GemmParams {
 // cg = 1: one CTA per 128 x 256 tile; cg = 2: a CTA pair per 256 x 256 tile.
 cudaError_t launch_gemm(int fmt, int epi, int cg, const GemmParams& p, int num_sms,
                         cudaStream_t st);
-int gemm_smem_bytes(int fmt, int cg);
+// N of the GEMM tile for a format / epilogue (the weight scale layout uses it).
+int gemm_tile_n(int fmt, int epi);
 
 // Error codes written to the device error word by the GEMM watchdog.
 enum : uint32_t { ERR_WAIT_PRODUCER = 1u, ERR_WAIT_MMA = 2u, ERR_WAIT_EPI = 4u };

@@ -124,7 +124,8 @@ ql_status quantize_act_noalloc(int fmt, int64_t K, int num_sms, const void* x, i
   reduce_amax_kernel<<<1, 256, 0, st>>>(scratch, nrb, scratch + kMaxRowBlocks);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess)
-    e = launch_quant_nvfp4(x, M, K, K, static_cast<uint8_t*>(codes), sf, 0, scratch + kMaxRowBlocks,
+    e = launch_quant_nvfp4(x, M, K, K, static_cast<uint8_t*>(codes), sf, 0, 128,
+                           scratch + kMaxRowBlocks,
                            g, RowMap{0, 0}, st);
   if (e != cudaSuccess) {
     cudaGetLastError();

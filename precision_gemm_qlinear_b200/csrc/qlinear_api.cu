@@ -38,6 +38,7 @@ struct qlinear_s {
   __nv_bfloat16* bias;
   RowMap map;
   int32_t fault_mode;  // test hook, see qlinear_debug_set_fault
+  int32_t bn;          // N of the GEMM tile (256, or 224 for NVFP4 without SwiGLU)
   CUtensorMap tmB1;    // weight codes, box 128 B x 256 rows (one CTA per tile)
   CUtensorMap tmB2;    // weight codes, box 128 B x 128 rows (CTA pair per tile)
   CUtensorMap tmSFB;   // NVFP4: weight SF atoms as 2048-byte rows (CTA pair)
@@ -65,7 +66,8 @@ WsLayout ws_layout(const ql_desc& d) {
                                               : static_cast<size_t>(d.N) * d.K;
   off = align_up(off + code_bytes, 1024);
   L.scales = off;
-  const size_t sc_bytes = d.fmt == QL_NVFP4 ? static_cast<size_t>(sfb_bytes(d.N, d.K)) + 16
+  const size_t sc_bytes = d.fmt == QL_NVFP4
+                              ? static_cast<size_t>(sfb_bytes(d.N, d.K, gemm_tile_n(d.fmt, d.epi))) + 16
                                             : static_cast<size_t>(d.N) * 4;
   off = align_up(off + sc_bytes, 1024);
   L.bias = off;
@@ -82,7 +84,7 @@ ql_status check_desc(const ql_desc* d) {
   if (d->N < 1 || d->K < 1 || d->N > (1 << 24) || d->K > (1 << 24)) return QL_ERR_INVALID_ARG;
   if (d->N % 32 != 0) return QL_ERR_INVALID_ARG;
   if (d->fmt == QL_FP8_E4M3 && d->K % 16 != 0) return QL_ERR_INVALID_ARG;
-  if (d->fmt == QL_NVFP4 && (d->K % 32 != 0 || d->N % 256 != 0)) return QL_ERR_INVALID_ARG;
+  if (d->fmt == QL_NVFP4 && d->K % 32 != 0) return QL_ERR_INVALID_ARG;
   if (d->epi == QL_EPI_SWIGLU && d->N % 256 != 0) return QL_ERR_INVALID_ARG;
   if (d->epi == QL_EPI_SPLIT_BIAS_GELU &&
       (d->split_col < 0 || d->split_col > d->N || d->split_col % 32 != 0))
@@ -234,6 +236,7 @@ ql_status qlinear_create(const ql_desc* desc, const void* w_bf16, const void* bi
   h->bias = reinterpret_cast<__nv_bfloat16*>(h->ws + L.bias);
   h->map.nout = h->Nout;
   h->map.mode = desc->epi == QL_EPI_SWIGLU ? 1 : 0;
+  h->bn = gemm_tile_n(desc->fmt, desc->epi);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   cudaError_t e = cudaMemsetAsync(h->ws, 0, 1024, st);
@@ -243,12 +246,14 @@ ql_status qlinear_create(const ql_desc* desc, const void* w_bf16, const void* bi
                               st);
   } else if (e == cudaSuccess) {
     h->wsf = h->ws + L.scales;
-    h->wG = reinterpret_cast<float*>(h->wsf + sfb_bytes(h->N, h->K));
+    h->wG = reinterpret_cast<float*>(h->wsf + sfb_bytes(h->N, h->K, h->bn));
     h->wamax = reinterpret_cast<uint32_t*>(h->wG + 1);
-    e = cudaMemsetAsync(h->wamax, 0, 4, st);
+    // unused scale words (rows past N, word 7 of a 224-row tile) stay zero
+    e = cudaMemsetAsync(h->wsf, 0, sfb_bytes(h->N, h->K, h->bn) + 16, st);
     if (e == cudaSuccess) e = launch_tensor_amax(w_bf16, h->N * h->K, h->wamax, h->num_sms, st);
     if (e == cudaSuccess)
-      e = launch_quant_nvfp4(w_bf16, h->N, h->K, h->K, h->wcodes, h->wsf, 1, h->wamax, h->wG, h->map,
+      e = launch_quant_nvfp4(w_bf16, h->N, h->K, h->K, h->wcodes, h->wsf, 1, h->bn, h->wamax, h->wG,
+                             h->map,
                              st);
   }
   if (e == cudaSuccess) e = launch_permute_bias(bias_bf16, h->bias, h->N, h->map, st);
@@ -259,11 +264,11 @@ ql_status qlinear_create(const ql_desc* desc, const void* w_bf16, const void* bi
   }
   const uint64_t kbytes = desc->fmt == QL_NVFP4 ? h->K / 2 : h->K;
   bool ok = make_tmap(&h->tmB1, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, 128,
-                      256, CU_TENSOR_MAP_SWIZZLE_128B) &&
+                      h->bn, CU_TENSOR_MAP_SWIZZLE_128B) &&
             make_tmap(&h->tmB2, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, 128,
-                      128, CU_TENSOR_MAP_SWIZZLE_128B);
+                      h->bn / 2, CU_TENSOR_MAP_SWIZZLE_128B);
   if (ok && desc->fmt == QL_NVFP4)
-    ok = make_sf_tmap(&h->tmSFB, h->wsf, sfb_bytes(h->N, h->K), 8);
+    ok = make_sf_tmap(&h->tmSFB, h->wsf, sfb_bytes(h->N, h->K, h->bn), 8);
   if (!ok) {
     delete h;
     return QL_ERR_CUDA;
@@ -303,7 +308,7 @@ ql_status qlinear_quantize_act(qlinear_t h, const void* x_bf16, int64_t M, void*
     e = cudaMemsetAsync(amax, 0, 4, st);
     if (e == cudaSuccess) e = launch_tensor_amax(x_bf16, M * h->K, amax, h->num_sms, st);
     if (e == cudaSuccess)
-      e = launch_quant_nvfp4(x_bf16, M, h->K, h->K, static_cast<uint8_t*>(codes), sf, 0, amax, g,
+      e = launch_quant_nvfp4(x_bf16, M, h->K, h->K, static_cast<uint8_t*>(codes), sf, 0, 128, amax, g,
                              RowMap{0, 0}, st);
   }
   if (e != cudaSuccess) cudaGetLastError();
@@ -367,7 +372,7 @@ ql_status qlinear_forward(qlinear_t h, const void* codes, const void* scales, in
   p.split_col = static_cast<int32_t>(h->d.split_col);
   p.k_blocks = static_cast<int32_t>((kbytes + 127) / 128);
   p.tiles_m = static_cast<int32_t>((M + 128 * cg - 1) / (128 * cg));
-  p.tiles_n = static_cast<int32_t>((h->N + 255) / 256);
+  p.tiles_n = static_cast<int32_t>((h->N + h->bn - 1) / h->bn);
   p.group_m = 8;
   p.sf_kchunks_a = static_cast<int32_t>(sf_kchunks(h->K));
   p.sfb_nstages = static_cast<int32_t>(sfb_stages(h->K));
@@ -408,7 +413,7 @@ ql_status qlinear_export_weights(qlinear_t h, void* codes_host, void* scales_hos
     float* sh = static_cast<float*>(scales_host);
     for (int64_t p = 0; p < h->N; ++p) sh[h->map(p)] = sc[p];
   } else {
-    std::vector<uint8_t> sf(sfb_bytes(h->N, h->K));
+    std::vector<uint8_t> sf(sfb_bytes(h->N, h->K, h->bn));
     float g = 0.f;
     if (cudaMemcpy(sf.data(), h->wsf, sf.size(), cudaMemcpyDeviceToHost) != cudaSuccess ||
         cudaMemcpy(&g, h->wG, 4, cudaMemcpyDeviceToHost) != cudaSuccess) {
@@ -419,7 +424,8 @@ ql_status qlinear_export_weights(qlinear_t h, void* codes_host, void* scales_hos
     uint8_t* sh = static_cast<uint8_t*>(scales_host);
     for (int64_t p = 0; p < h->N; ++p)
       for (int64_t b = 0; b < nb; ++b)
-        sh[h->map(p) * nb + b] = sf[sfb_word_offset(p, b / 16, (b / 4) & 3, 0, nks) + (b & 3)];
+        sh[h->map(p) * nb + b] =
+            sf[sfb_word_offset(p, b / 16, (b / 4) & 3, 0, nks, h->bn) + (b & 3)];
     if (global_scale) *global_scale = g;
   }
   return QL_OK;

@@ -154,7 +154,8 @@ __global__ void __launch_bounds__(256) tensor_amax_kernel(const uint4* __restric
 // padding scale is written as zero.
 __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
     const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K, int64_t ldx,
-    uint8_t* __restrict__ q, uint8_t* __restrict__ sf, int sf_layout, int64_t nks, int64_t mpad,
+    uint8_t* __restrict__ q, uint8_t* __restrict__ sf, int sf_layout, int64_t bn, int64_t nks,
+    int64_t mpad,
     const uint32_t* __restrict__ amax_bits, float* g_out, RowMap map) {
   const int64_t ngp = nks * 4;  // padded 64-element groups per row
   const int64_t nb = K >> 4;
@@ -192,7 +193,7 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
   } else {
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4)
-      *reinterpret_cast<uint32_t*>(sf + sfb_word_offset(row, g >> 2, g & 3, q4, nks)) = word;
+      *reinterpret_cast<uint32_t*>(sf + sfb_word_offset(row, g >> 2, g & 3, q4, nks, bn)) = word;
   }
 }
 
@@ -242,16 +243,16 @@ cudaError_t launch_tensor_amax(const void* x, int64_t n_elems, uint32_t* amax_bi
 }
 
 cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
-                               uint8_t* sf, int sf_layout, const uint32_t* amax_bits,
+                               uint8_t* sf, int sf_layout, int64_t bn, const uint32_t* amax_bits,
                                float* g_out, RowMap map, cudaStream_t st) {
-  // weights (layout 1) pad rows to the 256-row N tile, activations to 128
-  const int64_t mpad = sf_layout == 1 ? ((M + 255) / 256) * 256 : ((M + 127) / 128) * 128;
+  // weights (layout 1) pad rows to the N tile, activations to 128
+  const int64_t mpad = sf_layout == 1 ? ((M + bn - 1) / bn) * bn : ((M + 127) / 128) * 128;
   const int64_t nks = sfb_stages(K);  // == sf_kchunks(K) / 4
   const int64_t total = mpad * nks * 4;
   if (total <= 0) return cudaSuccess;
   const int64_t blocks = (total + 255) / 256;
   quant_nvfp4_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(x), M, K, ldx, q, sf, sf_layout, nks, mpad, amax_bits,
+      static_cast<const __nv_bfloat16*>(x), M, K, ldx, q, sf, sf_layout, bn, nks, mpad, amax_bits,
       g_out, map);
   return cudaGetLastError();
 }

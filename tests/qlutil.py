@@ -69,16 +69,17 @@ def sample_rows(M: int, n: int, seed: int = 0) -> np.ndarray:
 
 
 
-def sfb_word_offsets(N: int, K: int):
+def sfb_word_offsets(N: int, K: int, bn: int = 256):
     """Byte offset of the scale word of every (weight row n, stage ks, MMA step
-    j, replica q) in the replicated weight layout: per 256-row tile, stage and
+    j, replica q) in the replicated weight layout: per bn-row tile, stage and
     step a 4096-byte chunk of 128 rows x 32 bytes in core-matrix order; row
-    l = 32 q + n % 32, word (n % 256) // 32."""
+    l = 32 q + (n % bn) % 32, word (n % bn) // 32."""
     nks = (K + 255) // 256
-    n = np.arange(((N + 255) // 256) * 256)[:, None, None, None]
+    n = np.arange(((N + bn - 1) // bn) * bn)[:, None, None, None]
     ks = np.arange(nks)[None, :, None, None]
     j = np.arange(4)[None, None, :, None]
     q = np.arange(4)[None, None, None, :]
-    l = q * 32 + n % 32
-    w = (n % 256) // 32
-    return (((n // 256) * nks + ks) * 4 + j) * 4096 + (l // 8) * 256 + (w // 4) * 128 + (l % 8) * 16 + (w % 4) * 4
+    loc = n % bn
+    l = q * 32 + loc % 32
+    w = loc // 32
+    return (((n // bn) * nks + ks) * 4 + j) * 4096 + (l // 8) * 256 + (w // 4) * 128 + (l % 8) * 16 + (w % 4) * 4

@@ -35,3 +35,15 @@ def test_weight_sf_layout_words_tile_the_buffer(N, K):
     total = ((N + 255) // 256) * ((K + 255) // 256) * 4 * 4096
     assert np.all(off % 4 == 0)
     assert np.array_equal(np.sort(off), np.arange(0, total, 4))
+
+
+@pytest.mark.parametrize("N,K", [(224, 256), (768, 3072), (21504, 512)])
+def test_weight_sf_layout_224_row_tiles(N, K):
+    # 224-row tiles use words 0..6 of every row: the slots are distinct and
+    # the unused word 7 of each row is exactly what is left over
+    off = sfb_word_offsets(N, K, 224).ravel()
+    tiles = (N + 223) // 224
+    total = tiles * ((K + 255) // 256) * 4 * 4096
+    assert len(np.unique(off)) == off.size
+    assert off.size * 8 == total // 4 * 7
+    assert np.all(((off % 256) % 16 // 4 + 4 * ((off % 256) // 128)) != 7)
