@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--sets", type=int, default=0, help="input rotation sets (0 = auto)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override M of every layer (smaller captures for profiling only)")
     return ap.parse_args()
 
 
@@ -146,6 +148,15 @@ class ClockSampler:
         reasons = [k for k, v in self.REASONS.items() if self.reasons & v and k != "gpu_idle"]
         return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
                 "reasons": reasons, "samples": len(self.samples)}
+
+
+def with_tokens(wl, tokens):
+    """The workload with every layer's M replaced (0 = unchanged)."""
+    if not tokens:
+        return wl
+    import dataclasses
+    layers = tuple(dataclasses.replace(l, M=int(tokens)) for l in wl.layers)
+    return dataclasses.replace(wl, name=f"{wl.name}@M={tokens}", layers=layers)
 
 
 # ------------------------------------------------------- multi-rank helpers
@@ -262,10 +273,13 @@ def cpu_baseline(wl, seconds):
                         gate=inp.get("gate"), split_col=layer.split_col)
         return time.perf_counter() - t0
 
-    probe = 2
+    probe = 4
     t = run(probe)
+    while t < 0.5 and probe < layer.M:
+        probe = min(layer.M, probe * 4)
+        t = run(probe)
     rows = int(max(1, min(layer.M, probe * seconds / max(t, 1e-6))))
-    dt = run(rows)
+    dt = run(rows) if rows != probe else t
     flops = 2.0 * rows * layer.N * layer.K
     return flops / dt / 1e12, rows, dt, oracle.num_threads()
 
@@ -282,7 +296,7 @@ def main_ours(args):
                                 device_id=torch.device("cuda", local_rank))
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = WORKLOADS[args.workload]
+    wl = with_tokens(WORKLOADS[args.workload], args.tokens)
 
     per_set = 0
     for layer in wl.layers:
@@ -457,7 +471,18 @@ def main_reference(args):
         qa, sfa, ga = oracle.quant_nvfp4(x[:1], amax=amax)
         oracle.gemm_nvfp4(qa, sfa, ga, qw, sfw, gw)
     t1 = time.perf_counter() - t0
-    rows = int(max(1, min(layer.M, budget_s / max(t1, 1e-6))))
+    probe = 1
+    while t1 < 0.5 and probe < layer.M:  # size the per-step sample from a timed probe
+        probe = min(layer.M, probe * 4)
+        t0 = time.perf_counter()
+        if layer.fmt == "fp8":
+            qa, sa = oracle.quant_fp8_rows(x[:probe])
+            oracle.gemm_fp8(qa, sa, qw, sw)
+        else:
+            qa, sfa, ga = oracle.quant_nvfp4(x[:probe], amax=amax)
+            oracle.gemm_nvfp4(qa, sfa, ga, qw, sfw, gw)
+        t1 = time.perf_counter() - t0
+    rows = int(max(1, min(layer.M, probe * budget_s / max(t1, 1e-6))))
 
     def step(i):
         r0 = (i * rows) % max(1, layer.M - rows + 1)
