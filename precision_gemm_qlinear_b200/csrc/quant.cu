@@ -65,8 +65,11 @@ __device__ __forceinline__ uint4 ld_nc(const uint4* p) {
 // A team of T threads handles one row; 256 / T rows per CTA iteration.  Up to
 // VPL 16-byte vectors per thread stay in registers between the amax and the
 // cast; longer rows re-read the remainder (L2-resident by then).
+// __launch_bounds__(256, 4): at most 64 registers, so that four CTAs (32
+// warps) fit on an SM and a FLUX-sized activation (4608 rows of 3072 = 1152
+// CTAs of 4 rows) needs about two short waves with 16 rows in flight per SM.
 template <int T, int VPL>
-__global__ void __launch_bounds__(256) quant_fp8_rows_kernel(const __nv_bfloat16* __restrict__ x,
+__global__ void __launch_bounds__(256, 4) quant_fp8_rows_kernel(const __nv_bfloat16* __restrict__ x,
                                                              int64_t M, int64_t K, int64_t ldx,
                                                              uint8_t* __restrict__ q,
                                                              float* __restrict__ s, RowMap map) {
@@ -75,7 +78,7 @@ __global__ void __launch_bounds__(256) quant_fp8_rows_kernel(const __nv_bfloat16
   __shared__ uint32_t red[8];
   const int team = threadIdx.x / T;
   const int tt = threadIdx.x % T;
-  const int64_t nvec = K >> 3;
+  const int nvec = static_cast<int>(K >> 3);  // 16-byte vectors per row (K < 2^24)
   for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * TEAMS; row0 < M;
        row0 += static_cast<int64_t>(gridDim.x) * TEAMS) {
     const int64_t row = row0 + team;
@@ -85,13 +88,13 @@ __global__ void __launch_bounds__(256) quant_fp8_rows_kernel(const __nv_bfloat16
     float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      const int64_t idx = tt + static_cast<int64_t>(i) * T;
+      const int idx = tt + i * T;
       if (valid && idx < nvec) {
         v[i] = ld_nc(xr + idx);
         amax = fmaxf(amax, absmax8(v[i]));
       }
     }
-    for (int64_t idx = tt + static_cast<int64_t>(VPL) * T; valid && idx < nvec; idx += T)
+    for (int idx = tt + VPL * T; valid && idx < nvec; idx += T)
       amax = fmaxf(amax, absmax8(ld_nc(xr + idx)));
     // amax >= 0, so the float bit patterns order like unsigned integers
     uint32_t a = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
@@ -111,10 +114,10 @@ __global__ void __launch_bounds__(256) quant_fp8_rows_kernel(const __nv_bfloat16
     uint2* qr = reinterpret_cast<uint2*>(q + row * K);
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      const int64_t idx = tt + static_cast<int64_t>(i) * T;
+      const int idx = tt + i * T;
       if (valid && idx < nvec) qr[idx] = e4m3_8(v[i], inv);
     }
-    for (int64_t idx = tt + static_cast<int64_t>(VPL) * T; valid && idx < nvec; idx += T)
+    for (int idx = tt + VPL * T; valid && idx < nvec; idx += T)
       qr[idx] = e4m3_8(ld_nc(xr + idx), inv);
   }
 }
@@ -210,11 +213,11 @@ __global__ void permute_bias_kernel(const __nv_bfloat16* __restrict__ src,
 cudaError_t launch_quant_fp8_rows(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
                                   float* s, RowMap map, int num_sms, cudaStream_t st) {
   if (M <= 0) return cudaSuccess;
-  constexpr int VPL = 12;  // 96 bf16 per thread in registers
+  constexpr int VPL = 8;  // 64 bf16 per thread in registers
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   auto grid_for = [&](int teams) {
     int64_t blocks = (M + teams - 1) / teams;
-    int64_t cap = static_cast<int64_t>(num_sms) * 8;
+    int64_t cap = static_cast<int64_t>(num_sms) * 16;
     return static_cast<unsigned>(blocks < cap ? blocks : cap);
   };
   const int64_t per_warp = 32 * VPL * 8;
