@@ -175,6 +175,31 @@ __device__ __forceinline__ float silu_f(float g) {
   return g * rcp_newton(1.0f + ex2_sfu(x));
 }
 
+// Whole-chunk forms: each phase runs over all 32 independent elements of a
+// thread's chunk, so consecutive instructions do not depend on each other.
+__device__ __forceinline__ void gelu_tanh_32(float (&v)[32]) {
+  float d[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float t = fmaf(0.044715f * v[i], v[i], 1.0f);
+    d[i] = fminf(-2.3022081983953454f * v[i] * t, 126.0f);
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) d[i] = 1.0f + ex2_sfu(d[i]);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] *= rcp_newton(d[i]);
+}
+
+__device__ __forceinline__ void silu_mul_32(float (&g)[32], const float (&u)[32]) {
+  float d[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) d[i] = fminf(-1.4426950408889634f * g[i], 126.0f);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) d[i] = 1.0f + ex2_sfu(d[i]);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) g[i] = g[i] * rcp_newton(d[i]) * u[i];
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -528,50 +553,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
         const uint32_t* ra = acc[(EPI == EPI_SWIGLU) ? 0 : (ci & 1)];
         uint32_t packed[16];
         if (live) {
+          float v[32];
           if constexpr (EPI == EPI_SWIGLU) {
+            float u[32];
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              float o[2];
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                float sa_, sb_;
-                if constexpr (C::NV) {
-                  sa_ = rs;
-                  sb_ = rs;
-                } else {
-                  sa_ = rs * sw_a[i + h];
-                  sb_ = rs * sw_b[i + h];
-                }
-                const float g = fmaf(__uint_as_float(ra[i + h]), sa_, bf16x32_at(bias_a, i + h));
-                const float u = fmaf(__uint_as_float(accu[i + h]), sb_, bf16x32_at(bias_b, i + h));
-                o[h] = silu_f(g) * u;
+            for (int i = 0; i < 32; ++i) {
+              float sa_, sb_;
+              if constexpr (C::NV) {
+                sa_ = rs;
+                sb_ = rs;
+              } else {
+                sa_ = rs * sw_a[i];
+                sb_ = rs * sw_b[i];
               }
-              packed[i >> 1] = pack_bf16x2(o[0], o[1]);
+              v[i] = fmaf(__uint_as_float(ra[i]), sa_, bf16x32_at(bias_a, i));
+              u[i] = fmaf(__uint_as_float(accu[i]), sb_, bf16x32_at(bias_b, i));
             }
+            silu_mul_32(v, u);
           } else {
-            const bool gelu_chunk =
-                (EPI == EPI_BIAS_GELU) || (EPI == EPI_SPLIT && ncol >= p.split_col);
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              float o[2];
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                float s_;
-                if constexpr (C::NV)
-                  s_ = rs;
-                else
-                  s_ = rs * sw_a[i + h];
-                float v = fmaf(__uint_as_float(ra[i + h]), s_, bf16x32_at(bias_a, i + h));
-                if constexpr (EPI == EPI_GATED_RES)
-                  v = fmaf(bf16x32_at(gate_a, i + h), v, bf16x32_at(res_a, i + h));
-                if constexpr (EPI == EPI_BIAS_GELU || EPI == EPI_SPLIT) {
-                  if (gelu_chunk) v = gelu_tanh_f(v);
-                }
-                o[h] = v;
-              }
-              packed[i >> 1] = pack_bf16x2(o[0], o[1]);
+            for (int i = 0; i < 32; ++i) {
+              float s_;
+              if constexpr (C::NV)
+                s_ = rs;
+              else
+                s_ = rs * sw_a[i];
+              v[i] = fmaf(__uint_as_float(ra[i]), s_, bf16x32_at(bias_a, i));
+              if constexpr (EPI == EPI_GATED_RES)
+                v[i] = fmaf(bf16x32_at(gate_a, i), v[i], bf16x32_at(res_a, i));
+            }
+            if constexpr (EPI == EPI_BIAS_GELU) {
+              gelu_tanh_32(v);
+            } else if constexpr (EPI == EPI_SPLIT) {
+              if (ncol >= p.split_col) gelu_tanh_32(v);  // uniform per chunk
             }
           }
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) packed[i >> 1] = pack_bf16x2(v[i], v[i + 1]);
         }
         if constexpr (EPI == EPI_SWIGLU) {
           // SwiGLU holds two halves per chunk; the next pair is loaded here,
