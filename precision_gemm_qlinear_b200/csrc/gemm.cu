@@ -292,6 +292,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
     __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sb->tmem_base;
+  // everything above overlapped the tail of the kernel that produced the
+  // activation codes and scales; from here on they are read
+  grid_dep_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
@@ -624,6 +627,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
   }
 
   __syncwarp();
+  grid_dep_launch_dependents();
   tc_fence_before();
   if constexpr (C::PAIR)
     cluster_sync_all();  // no CTA leaves while its peer may still signal its barriers
@@ -658,13 +662,15 @@ cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t st) {
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CG;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 

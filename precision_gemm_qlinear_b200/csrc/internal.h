@@ -62,6 +62,23 @@ __host__ __device__ __forceinline__ int64_t sfb_word_offset(int64_t n, int64_t k
          (w & 3) * 4;
 }
 
+// Launch configuration with programmatic stream serialization: the kernel may
+// start while the previous kernel in the stream finishes; it calls
+// grid_dep_wait() before touching anything that kernel produced.
+inline cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                     cudaLaunchAttribute* attrs, unsigned nattrs_before) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  attrs[nattrs_before].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[nattrs_before].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = nattrs_before + 1;
+  return cfg;
+}
+
 // -------------------------------------------------------------- quantize
 
 cudaError_t launch_quant_fp8_rows(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
@@ -96,6 +113,7 @@ struct alignas(64) GemmParams {
   const __nv_bfloat16* bias;      // [N] (zeros when the layer has no bias)
   const __nv_bfloat16* residual;  // [M, Nout] or null
   const __nv_bfloat16* gate;      // [Nout] or null
+  __nv_bfloat16* out;             // [M, Nout] (the TMA store map tmC covers the same buffer)
   uint32_t* err;          // device error word of the handle
   int32_t M, N, Nout, split_col;
   int32_t k_blocks;       // number of 128-byte K stages

@@ -365,6 +365,7 @@ ql_status qlinear_forward(qlinear_t h, const void* codes, const void* scales, in
   p.bias = h->bias;
   p.residual = static_cast<const __nv_bfloat16*>(residual);
   p.gate = static_cast<const __nv_bfloat16*>(gate);
+  p.out = static_cast<__nv_bfloat16*>(out_bf16);
   p.err = h->err;
   p.M = static_cast<int32_t>(M);
   p.N = static_cast<int32_t>(h->N);

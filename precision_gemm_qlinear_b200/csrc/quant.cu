@@ -79,6 +79,8 @@ __global__ void __launch_bounds__(256, 4) quant_fp8_rows_kernel(const __nv_bfloa
   const int team = threadIdx.x / T;
   const int tt = threadIdx.x % T;
   const int nvec = static_cast<int>(K >> 3);  // 16-byte vectors per row (K < 2^24)
+  grid_dep_wait();               // x may come from the previous kernel
+  grid_dep_launch_dependents();  // the GEMM may start its prologue
   for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * TEAMS; row0 < M;
        row0 += static_cast<int64_t>(gridDim.x) * TEAMS) {
     const int64_t row = row0 + team;
@@ -126,6 +128,8 @@ __global__ void __launch_bounds__(256, 4) quant_fp8_rows_kernel(const __nv_bfloa
 
 __global__ void __launch_bounds__(256) tensor_amax_kernel(const uint4* __restrict__ x,
                                                           int64_t nvec, uint32_t* amax_bits) {
+  grid_dep_wait();
+  grid_dep_launch_dependents();
   float m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -165,6 +169,8 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t row = idx / ngp;
   const int64_t g = idx - row * ngp;
+  grid_dep_wait();  // the tensor amax of the previous kernel
+  grid_dep_launch_dependents();
   if (row >= mpad) return;
   const float A = __uint_as_float(*amax_bits);
   const float G = __fdiv_rn(A, 2688.f);
@@ -221,16 +227,19 @@ cudaError_t launch_quant_fp8_rows(const void* x, int64_t M, int64_t K, int64_t l
     return static_cast<unsigned>(blocks < cap ? blocks : cap);
   };
   const int64_t per_warp = 32 * VPL * 8;
+  cudaLaunchAttribute at[1];
   if (K <= per_warp) {
-    quant_fp8_rows_kernel<32, VPL><<<grid_for(8), 256, 0, st>>>(xb, M, K, ldx, q, s, map);
+    cudaLaunchConfig_t c = pdl_config(grid_for(8), 256, 0, st, at, 0);
+    return cudaLaunchKernelEx(&c, quant_fp8_rows_kernel<32, VPL>, xb, M, K, ldx, q, s, map);
   } else if (K <= 2 * per_warp) {
-    quant_fp8_rows_kernel<64, VPL><<<grid_for(4), 256, 0, st>>>(xb, M, K, ldx, q, s, map);
+    cudaLaunchConfig_t c = pdl_config(grid_for(4), 256, 0, st, at, 0);
+    return cudaLaunchKernelEx(&c, quant_fp8_rows_kernel<64, VPL>, xb, M, K, ldx, q, s, map);
   } else if (K <= 4 * per_warp) {
-    quant_fp8_rows_kernel<128, VPL><<<grid_for(2), 256, 0, st>>>(xb, M, K, ldx, q, s, map);
-  } else {
-    quant_fp8_rows_kernel<256, VPL><<<grid_for(1), 256, 0, st>>>(xb, M, K, ldx, q, s, map);
+    cudaLaunchConfig_t c = pdl_config(grid_for(2), 256, 0, st, at, 0);
+    return cudaLaunchKernelEx(&c, quant_fp8_rows_kernel<128, VPL>, xb, M, K, ldx, q, s, map);
   }
-  return cudaGetLastError();
+  cudaLaunchConfig_t c = pdl_config(grid_for(1), 256, 0, st, at, 0);
+  return cudaLaunchKernelEx(&c, quant_fp8_rows_kernel<256, VPL>, xb, M, K, ldx, q, s, map);
 }
 
 cudaError_t launch_tensor_amax(const void* x, int64_t n_elems, uint32_t* amax_bits, int num_sms,
@@ -240,9 +249,9 @@ cudaError_t launch_tensor_amax(const void* x, int64_t n_elems, uint32_t* amax_bi
   int64_t blocks = (nvec + 255) / 256;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   if (blocks > cap) blocks = cap;
-  tensor_amax_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      static_cast<const uint4*>(x), nvec, amax_bits);
-  return cudaGetLastError();
+  cudaLaunchAttribute at[1];
+  cudaLaunchConfig_t c = pdl_config(static_cast<unsigned>(blocks), 256, 0, st, at, 0);
+  return cudaLaunchKernelEx(&c, tensor_amax_kernel, static_cast<const uint4*>(x), nvec, amax_bits);
 }
 
 cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
@@ -254,10 +263,10 @@ cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx,
   const int64_t total = mpad * nks * 4;
   if (total <= 0) return cudaSuccess;
   const int64_t blocks = (total + 255) / 256;
-  quant_nvfp4_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(x), M, K, ldx, q, sf, sf_layout, bn, nks, mpad, amax_bits,
-      g_out, map);
-  return cudaGetLastError();
+  cudaLaunchAttribute at[1];
+  cudaLaunchConfig_t c = pdl_config(static_cast<unsigned>(blocks), 256, 0, st, at, 0);
+  return cudaLaunchKernelEx(&c, quant_nvfp4_kernel, static_cast<const __nv_bfloat16*>(x), M, K,
+                            ldx, q, sf, sf_layout, bn, nks, mpad, amax_bits, g_out, map);
 }
 
 cudaError_t launch_permute_bias(const void* src, void* dst, int64_t N, RowMap map,
