@@ -110,6 +110,7 @@ struct SmemBars {
   uint32_t tmem_base;
   volatile int32_t abort_flag;
 };
+static_assert(sizeof(SmemBars) <= 256, "barrier block exceeds its reservation");
 
 __device__ __forceinline__ void tile_coords(int t, const GemmParams& p, int& mb, int& nb) {
   const int per_group = p.group_m * p.tiles_n;
@@ -142,62 +143,50 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, SmemBar
   }
 }
 
-// The GELU / SiLU epilogues are bound by the special-function unit, so each
-// element uses exactly one SFU operation (the base-2 exponential) and takes
-// the reciprocal on the FMA pipe: Newton-Raphson r <- r (2 - d r) from the
-// classic exponent-bit initial guess, three steps (relative error < 2e-7 for
-// d >= 1).
+// GELU and SiLU take two special-function-unit operations per element (the
+// base-2 exponential and the reciprocal).  The epilogue warps share their
+// schedulers with the MMA-issuing thread, so issue slots are the scarce
+// resource there; the SFU itself stays lightly loaded (two operations per
+// element at 16 lanes per clock per SM is well under the tile time).
 __device__ __forceinline__ float ex2_sfu(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-__device__ __forceinline__ float rcp_newton(float d) {  // d >= 1, finite
-  float r = __int_as_float(0x7EF311C7 - __float_as_int(d));
-  r = r * fmaf(-d, r, 2.0f);
-  r = r * fmaf(-d, r, 2.0f);
-  r = r * fmaf(-d, r, 2.0f);
+__device__ __forceinline__ float rcp_sfu(float d) {  // d >= 1; rcp(+inf) = +0
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));
   return r;
 }
 
-__device__ __forceinline__ float gelu_tanh_f(float v) {
-  // 0.5 v (1 + tanh(u)) = v / (1 + e^{-2u}), u = sqrt(2/pi) v (1 + 0.044715 v^2);
-  // e^{-2u} = 2^{-2 u log2(e)}; the exponent is clamped so 1 + e stays finite
-  const float t = fmaf(0.044715f * v, v, 1.0f);
-  const float x = fminf(-2.3022081983953454f * v * t, 126.0f);  // -2 sqrt(2/pi) log2(e)
-  return v * rcp_newton(1.0f + ex2_sfu(x));
-}
-
-__device__ __forceinline__ float silu_f(float g) {
-  // g / (1 + e^{-g}),  e^{-g} = 2^{-g log2(e)}
-  const float x = fminf(-1.4426950408889634f * g, 126.0f);
-  return g * rcp_newton(1.0f + ex2_sfu(x));
-}
+// GELU-tanh: 0.5 v (1 + tanh(u)) = v / (1 + e^{-2u}), u = sqrt(2/pi) (v + 0.044715 v^3),
+// and e^{-2u} = 2^{v (A + B v^2)} with A = -2 sqrt(2/pi) log2(e), B = 0.044715 A.
+// SiLU: g / (1 + e^{-g}), e^{-g} = 2^{-g log2(e)}.  For very negative inputs
+// the exponential overflows to +inf and the reciprocal returns 0, which is the
+// limit of both functions, so no clamp is needed.
+constexpr float kGeluA = -2.302208198144325f;
+constexpr float kGeluB = -0.1029432395800235f;
+constexpr float kNegLog2e = -1.4426950408889634f;
 
 // Whole-chunk forms: each phase runs over all 32 independent elements of a
 // thread's chunk, so consecutive instructions do not depend on each other.
 __device__ __forceinline__ void gelu_tanh_32(float (&v)[32]) {
   float d[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const float t = fmaf(0.044715f * v[i], v[i], 1.0f);
-    d[i] = fminf(-2.3022081983953454f * v[i] * t, 126.0f);
-  }
+  for (int i = 0; i < 32; ++i) d[i] = v[i] * fmaf(kGeluB, v[i] * v[i], kGeluA);
 #pragma unroll
   for (int i = 0; i < 32; ++i) d[i] = 1.0f + ex2_sfu(d[i]);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] *= rcp_newton(d[i]);
+  for (int i = 0; i < 32; ++i) v[i] *= rcp_sfu(d[i]);
 }
 
 __device__ __forceinline__ void silu_mul_32(float (&g)[32], const float (&u)[32]) {
   float d[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) d[i] = fminf(-1.4426950408889634f * g[i], 126.0f);
+  for (int i = 0; i < 32; ++i) d[i] = 1.0f + ex2_sfu(kNegLog2e * g[i]);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) d[i] = 1.0f + ex2_sfu(d[i]);
-#pragma unroll
-  for (int i = 0; i < 32; ++i) g[i] = g[i] * rcp_newton(d[i]) * u[i];
+  for (int i = 0; i < 32; ++i) g[i] = g[i] * rcp_sfu(d[i]) * u[i];
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -383,6 +372,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
       bool ok = true;
       bool any = false;
       int local = 0;
+      // The issuing thread shares its scheduler with two epilogue warps, so
+      // everything that does not change from stage to stage is computed once:
+      // stage-0 operand and scale descriptors, scale-factor TMEM addresses.
+      const uint32_t s0 = smem_u32(smem);
+      const uint64_t d_a0 = sdesc_k_sw128(s0);
+      const uint64_t d_b0 = sdesc_k_sw128(s0 + A_BYTES);
+      const uint64_t d_sfa0 = sdesc_k_interleave(s0 + A_BYTES + C::B_BYTES);
+      const uint64_t d_sfb0 = sdesc_k_interleave2(s0 + A_BYTES + C::B_BYTES + C::SFA_BYTES, 128, 256);
+      const uint32_t t_sfa = tmem + C::SFA_COL;
+      const uint32_t t_sfb = tmem + C::SFB_COL;
       for (int t = unit; t < num_tiles && ok; t += nunits, ++local) {
         const int buf = local & 1;
         const uint32_t use = static_cast<uint32_t>(local >> 1);
@@ -399,39 +398,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
             break;
           }
           tc_fence_after();
-          uint8_t* st = smem + stage * C::STAGE_BYTES;
-          const uint32_t a_addr = smem_u32(st);
-          const uint32_t b_addr = smem_u32(st + A_BYTES);
+          // this stage's descriptors: the stage-0 descriptors advanced by the
+          // stage offset in the 16-byte start-address field
+          const uint64_t so = static_cast<uint64_t>(stage) * (C::STAGE_BYTES >> 4);
           if constexpr (C::NV) {
-            const uint32_t sfs = smem_u32(st + A_BYTES + C::B_BYTES);
             // per MMA step j: the A atom (32 x 128-bit, replicated to the 4
             // sub-partitions by the copy) and the pre-replicated B chunk
             // (128 x 256-bit)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const uint64_t da = sdesc_k_interleave(sfs + 512 * j);
-              const uint64_t db = sdesc_k_interleave2(sfs + C::SFA_BYTES + 4096 * j, 128, 256);
+              const uint64_t da = d_sfa0 + so + (512 >> 4) * j;
+              const uint64_t db = d_sfb0 + so + (4096 >> 4) * j;
               if constexpr (C::PAIR) {
-                tc_cp_32x128b_warpx4_pair(tmem + C::SFA_COL + 4 * j, da);
-                tc_cp_128x256b_pair(tmem + C::SFB_COL + 8 * j, db);
+                tc_cp_32x128b_warpx4_pair(t_sfa + 4 * j, da);
+                tc_cp_128x256b_pair(t_sfb + 8 * j, db);
               } else {
-                tc_cp_32x128b_warpx4(tmem + C::SFA_COL + 4 * j, da);
-                tc_cp_128x256b(tmem + C::SFB_COL + 8 * j, db);
+                tc_cp_32x128b_warpx4(t_sfa + 4 * j, da);
+                tc_cp_128x256b(t_sfb + 8 * j, db);
               }
             }
           }
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint64_t ad = sdesc_k_sw128(a_addr + 32 * j);
-            const uint64_t bd = sdesc_k_sw128(b_addr + 32 * j);
+            const uint64_t ad = d_a0 + so + (32 >> 4) * j;
+            const uint64_t bd = d_b0 + so + (32 >> 4) * j;
             const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
             if constexpr (C::NV) {
               if constexpr (C::PAIR)
-                mma_mxf4nvf4_pair(d_tmem, ad, bd, idesc_f4<CG, BN>(), tmem + C::SFA_COL + 4 * j,
-                                  tmem + C::SFB_COL + 8 * j, acc);
+                mma_mxf4nvf4_pair(d_tmem, ad, bd, idesc_f4<CG, BN>(), t_sfa + 4 * j, t_sfb + 8 * j,
+                                  acc);
               else
-                mma_mxf4nvf4(d_tmem, ad, bd, idesc_f4<CG, BN>(), tmem + C::SFA_COL + 4 * j,
-                             tmem + C::SFB_COL + 8 * j, acc);
+                mma_mxf4nvf4(d_tmem, ad, bd, idesc_f4<CG, BN>(), t_sfa + 4 * j, t_sfb + 8 * j,
+                             acc);
             } else {
               if constexpr (C::PAIR)
                 mma_f8f6f4_pair(d_tmem, ad, bd, idesc_f8<CG, BN>(), acc);
