@@ -113,12 +113,7 @@ QL_API ql_status qlinear_create(const ql_desc* desc, const void* w_bf16, const v
  *   NVFP4: codes [M, K/2] bytes (two codes per byte, low nibble first);
  *          scales = block scales in the GEMM's tiled layout
  *          (ceil(M/128) x ceil(K/256)*4 chunks of 512 bytes) followed by a
- *          16-byte tail holding the fp32 global scale and the amax word.
- *          Chunk c of row block R holds the scales of rows 128R..128R+127 for
- *          K elements 64c..64c+63; row r, block j has atom index
- *          a = (r%32)*16 + (r%128/32)*4 + j, and chunks 2i, 2i+1 are stored
- *          as one 1 KB unit interleaved in 128-byte pieces (byte
- *          (a/128)*256 + (c%2)*128 + a%128 of the unit). */
+ *          16-byte tail holding the fp32 global scale and the amax word. */
 QL_API ql_status qlinear_act_bytes(qlinear_t h, int64_t M, size_t* code_bytes, size_t* scale_bytes);
 
 /* Number of output columns of qlinear_forward (N, or N/2 for SwiGLU). */

@@ -75,16 +75,13 @@ struct Cfg {
   // in the 512 columns side by side.
   static constexpr int BN = (NV && EPI != EPI_SWIGLU) ? 224 : 256;
   static constexpr int B_BYTES = (BN / CG) * BK_BYTES;  // this CTA's rows of B
-  static constexpr int SFA_BYTES = NV ? 8192 : 0;       // 2 atom pairs x 4 replicas of 1 KB
+  static constexpr int SFA_BYTES = NV ? 2048 : 0;       // 4 atoms (one per MMA K step)
   static constexpr int SFB_BYTES = NV ? 16384 : 0;      // 4 replicated 4 KB chunks (all 256 B rows)
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int STAGES = NV ? (PAIR ? 4 : 3) : (PAIR ? 6 : 4);
-  // staging buffers per epilogue warp: two, one, or none (direct stores from
-  // registers) -- as many as the shared-memory budget leaves room for
-  static constexpr bool fits(int nbuf) {
-    return STAGES * STAGE_BYTES + NUM_EPI_WARPS * nbuf * STAGING_BYTES + 256 + 1024 <= 232448;
-  }
-  static constexpr int NBUF = fits(2) ? 2 : (fits(1) ? 1 : 0);
+  // staging buffers per epilogue warp: two unless that breaks the budget
+  static constexpr int NBUF =
+      (STAGES * STAGE_BYTES + NUM_EPI_WARPS * 2 * STAGING_BYTES + 256 + 1024 <= 232448) ? 2 : 1;
   static constexpr int STAGING_OFF = STAGES * STAGE_BYTES;
   static constexpr int BAR_OFF = STAGING_OFF + NUM_EPI_WARPS * NBUF * STAGING_BYTES;
   static_assert(BAR_OFF + 256 + 1024 <= 232448, "shared memory budget");
@@ -322,18 +319,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
               tma_load_2d_pair(smem_u32(st), &p.tmA, lfb, kb * BK_BYTES, a_row);
               tma_load_2d_pair(smem_u32(st + A_BYTES), &p.tmB, lfb, kb * BK_BYTES, b_row);
               if constexpr (C::NV) {
-                // scales through 2-D maps: the two A atom pairs of this CTA's
-                // 128 rows (1 KB rows of the map), each loaded four times to
-                // form the replicated source of one 128 x 256-bit copy; and
-                // the pre-replicated B chunks of the whole tile (8 rows of
-                // 2 KB; both CTAs need them)
+                // scales through 2-D maps of 2048-byte rows (uint64 x 256): the
+                // A atoms of this CTA's 128 rows (one row of the map) and the
+                // replicated B chunks of all 256 columns of the tile (8 rows;
+                // both CTAs need them)
                 const uint32_t sfs = smem_u32(st + A_BYTES + C::B_BYTES);
-                const int arow = ((mb * 2 + static_cast<int>(rank)) * p.sf_kchunks_a >> 1) + kb * 2;
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-#pragma unroll
-                  for (int r = 0; r < 4; ++r)
-                    tma_load_2d_pair(sfs + 4096 * c + 1024 * r, &p.tmSFA, lfb, 0, arow + c);
+                const int ka = p.sf_kchunks_a >> 2;
+                tma_load_2d_pair(sfs, &p.tmSFA, lfb, 0, (mb * 2 + static_cast<int>(rank)) * ka + kb);
                 tma_load_2d_pair(sfs + C::SFA_BYTES, &p.tmSFB, lfb, 0,
                                  8 * (nb * p.sfb_nstages + kb));
               }
@@ -347,10 +339,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
                 const uint8_t* sfb =
                     p.sfb + (static_cast<int64_t>(nb) * p.sfb_nstages + kb) * C::SFB_BYTES;
                 const uint32_t sfs = smem_u32(st + A_BYTES + C::B_BYTES);
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-#pragma unroll
-                  for (int r = 0; r < 4; ++r) bulk_load(sfs + 4096 * c + 1024 * r, sfa + 1024 * c, 1024, fb);
+                bulk_load(sfs, sfa, C::SFA_BYTES, fb);
                 bulk_load(sfs + C::SFA_BYTES, sfb, C::SFB_BYTES, fb);
               }
             }
@@ -389,7 +378,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
       const uint32_t s0 = smem_u32(smem);
       const uint64_t d_a0 = sdesc_k_sw128(s0);
       const uint64_t d_b0 = sdesc_k_sw128(s0 + A_BYTES);
-      const uint64_t d_sfa0 = sdesc_k_interleave2(s0 + A_BYTES + C::B_BYTES, 128, 256);
+      const uint64_t d_sfa0 = sdesc_k_interleave(s0 + A_BYTES + C::B_BYTES);
       const uint64_t d_sfb0 = sdesc_k_interleave2(s0 + A_BYTES + C::B_BYTES + C::SFA_BYTES, 128, 256);
       const uint32_t t_sfa = tmem + C::SFA_COL;
       const uint32_t t_sfb = tmem + C::SFB_COL;
@@ -413,24 +402,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
           // stage offset in the 16-byte start-address field
           const uint64_t so = static_cast<uint64_t>(stage) * (C::STAGE_BYTES >> 4);
           if constexpr (C::NV) {
-            // 128 x 256-bit copies from pre-replicated sources: A scales of
-            // two MMA steps per copy (8 columns, step j at t_sfa + 4 j), B
-            // scales of one step per copy (8 columns at t_sfb + 8 j)
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              const uint64_t da = d_sfa0 + so + (4096 >> 4) * c;
-              if constexpr (C::PAIR)
-                tc_cp_128x256b_pair(t_sfa + 8 * c, da);
-              else
-                tc_cp_128x256b(t_sfa + 8 * c, da);
-            }
+            // per MMA step j: the A atom (32 x 128-bit, replicated to the 4
+            // sub-partitions by the copy) and the pre-replicated B chunk
+            // (128 x 256-bit)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
+              const uint64_t da = d_sfa0 + so + (512 >> 4) * j;
               const uint64_t db = d_sfb0 + so + (4096 >> 4) * j;
-              if constexpr (C::PAIR)
+              if constexpr (C::PAIR) {
+                tc_cp_32x128b_warpx4_pair(t_sfa + 4 * j, da);
                 tc_cp_128x256b_pair(t_sfb + 8 * j, db);
-              else
+              } else {
+                tc_cp_32x128b_warpx4(t_sfa + 4 * j, da);
                 tc_cp_128x256b(t_sfb + 8 * j, db);
+              }
             }
           }
 #pragma unroll
@@ -617,35 +602,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
           }
         }
         if (!live) continue;
-        if constexpr (C::NBUF == 0) {
-          // no room for staging: each lane writes its row's 64 bytes
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(m) * p.Nout + ocol);
+        // ---- stage through swizzled shared memory, then one TMA store per warp
+        uint8_t* sbuf = staging + (nstore % C::NBUF) * STAGING_BYTES;
+        if (lane == 0) bulk_wait_group_read<C::NBUF - 1>();
+        __syncwarp();
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
-                                  packed[4 * j + 3]);
-          }
-          continue;
-        } else {
-          // ---- stage through swizzled shared memory, then one TMA store per warp
-          uint8_t* sbuf = staging + (nstore % C::NBUF) * STAGING_BYTES;
-          if (lane == 0) bulk_wait_group_read<C::NBUF - 1>();
-          __syncwarp();
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int sw = (j ^ ((lane >> 1) & 3)) << 4;
-            *reinterpret_cast<uint4*>(sbuf + lane * 64 + sw) =
-                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && slab_ok) {
-            tma_store_2d(&p.tmC, smem_u32(sbuf), ocol, row0);
-            bulk_commit_group();
-          }
-          ++nstore;
+        for (int j = 0; j < 4; ++j) {
+          const int sw = (j ^ ((lane >> 1) & 3)) << 4;
+          *reinterpret_cast<uint4*>(sbuf + lane * 64 + sw) =
+              make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && slab_ok) {
+          tma_store_2d(&p.tmC, smem_u32(sbuf), ocol, row0);
+          bulk_commit_group();
+        }
+        ++nstore;
       }
     }
     if (lane == 0) bulk_wait_group<0>();

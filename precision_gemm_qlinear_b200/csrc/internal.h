@@ -22,26 +22,17 @@ struct RowMap {
   }
 };
 
-// Scale-factor layout of the block-scaled GEMM's A operand (activations):
-// for a [rows, K] NVFP4 operand with one E4M3 scale per 16 K-elements, rows
-// are grouped in blocks of 128 and K in chunks of 64 (4 scales, one MMA step).
-// The scales of one (row block, K chunk) form a 512-byte atom in which row r
-// (0..127) and K-block j (0..3) have index a = (r % 32) * 16 + (r / 32) * 4 + j:
-// lane r % 32 of a 32 x 128-bit matrix whose four 32-bit columns are the four
-// 32-row groups.  Two consecutive atoms (K chunks 2c, 2c+1) are stored as one
-// 1 KB pair, interleaved in 128-byte pieces: piece p of the pair holds bytes
-// [128 p, 128 p + 128) of the even atom, then the same bytes of the odd atom.
-// Four copies of a pair side by side are exactly the shared-memory source of
-// one 128 x 256-bit tcgen05.cp that gives every TMEM sub-partition both
-// steps' scales.  Pairs are stored K fastest; the number of K chunks per row
-// block is padded to a multiple of 4 (one pipeline stage of 256 K-elements),
-// padding scales are 0.
+// Scale-factor layout of the block-scaled GEMM ("SF atoms"): for a [rows, K]
+// NVFP4 operand with one E4M3 scale per 16 K-elements, rows are grouped in
+// blocks of 128 and K in chunks of 64 (4 scales).  Each (row block, K chunk)
+// is a 512-byte atom; inside it the scale of row r (0..127) and K-block j
+// (0..3) sits at byte (r % 32) * 16 + (r / 32) * 4 + j.  Atoms are stored
+// K-chunk fastest; the number of K chunks per row block is padded to a
+// multiple of 4 (one pipeline stage of 256 K-elements), padding scales are 0.
 __host__ __device__ __forceinline__ int64_t sf_kchunks(int64_t K) { return ((K + 255) / 256) * 4; }
 __host__ __device__ __forceinline__ int64_t sf_offset(int64_t row, int64_t kb, int64_t kchunks) {
-  const int64_t a = (row & 31) * 16 + ((row & 127) >> 5) * 4 + (kb & 3);  // index in the atom
-  const int64_t chunk = kb >> 2;
-  return ((row >> 7) * kchunks + (chunk & ~static_cast<int64_t>(1))) * 512 + (a >> 7) * 256 +
-         (chunk & 1) * 128 + (a & 127);
+  return ((row >> 7) * kchunks + (kb >> 2)) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 +
+         (kb & 3);
 }
 __host__ __device__ __forceinline__ int64_t sf_bytes(int64_t rows, int64_t K) {
   return ((rows + 127) / 128) * sf_kchunks(K) * 512;
@@ -111,7 +102,7 @@ struct alignas(64) GemmParams {
   CUtensorMap tmA;  // activation codes [M, K(/2)] bytes, box 128 x 128 B, 128B swizzle
   CUtensorMap tmB;  // weight codes [N, K(/2)] bytes, box 128 B x (256 / CG) rows, 128B swizzle
   CUtensorMap tmC;  // output [M, Nout] bf16, box 32 x 32, 64B swizzle
-  CUtensorMap tmSFA;  // NVFP4 pair mode: activation SF as rows of 1 KB (one atom pair)
+  CUtensorMap tmSFA;  // NVFP4 pair mode: activation SF atoms as rows of 2048 bytes
   CUtensorMap tmSFB;  // NVFP4 pair mode: weight SF chunks as rows of 2048 bytes
   const float* sa;        // FP8: per-row activation scale [M]
   const float* sw;        // FP8: per-column weight scale [N]

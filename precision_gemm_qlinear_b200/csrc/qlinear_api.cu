@@ -157,15 +157,12 @@ bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
   return r == CUDA_SUCCESS;
 }
 
-// Scale-factor buffers viewed as rows of `row_bytes` bytes (uint64 elements),
-// box = one row wide and `box_rows` rows high.  Activation scales: rows of
-// 1 KB, one atom pair, boxes of 1 row.  Weight chunks: rows of 2 KB, boxes of
-// 8 rows = one stage of one N tile.
-bool make_sf_tmap(CUtensorMap* m, const void* base, int64_t bytes, int64_t row_bytes,
-                  uint32_t box_rows) {
-  const int64_t elems = row_bytes / 8;
-  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, base, elems, bytes / row_bytes, row_bytes,
-                   static_cast<uint32_t>(elems), box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
+// Scale-factor buffers viewed as rows of 2048 bytes: uint64 elements, 256 per
+// row, box = `box_rows` rows (activation atoms: 1 row = one pipeline stage of
+// one 128-row block; weight chunks: 8 rows = one stage of one 256-row tile).
+bool make_sf_tmap(CUtensorMap* m, const void* base, int64_t bytes, uint32_t box_rows) {
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, base, 256, bytes / 2048, 2048, 256,
+                   box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 ql_status from_cuda(cudaError_t e) {
@@ -271,7 +268,7 @@ ql_status qlinear_create(const ql_desc* desc, const void* w_bf16, const void* bi
             make_tmap(&h->tmB2, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, 128,
                       h->bn / 2, CU_TENSOR_MAP_SWIZZLE_128B);
   if (ok && desc->fmt == QL_NVFP4)
-    ok = make_sf_tmap(&h->tmSFB, h->wsf, sfb_bytes(h->N, h->K, h->bn), 2048, 8);
+    ok = make_sf_tmap(&h->tmSFB, h->wsf, sfb_bytes(h->N, h->K, h->bn), 8);
   if (!ok) {
     delete h;
     return QL_ERR_CUDA;
@@ -353,7 +350,7 @@ ql_status qlinear_forward(qlinear_t h, const void* codes, const void* scales, in
     return QL_ERR_CUDA;
   p.tmB = cg == 2 ? h->tmB2 : h->tmB1;
   if (nv && cg == 2) {
-    if (!make_sf_tmap(&p.tmSFA, scales, sf_bytes(M, h->K), 1024, 1)) return QL_ERR_CUDA;
+    if (!make_sf_tmap(&p.tmSFA, scales, sf_bytes(M, h->K), 1)) return QL_ERR_CUDA;
     p.tmSFB = h->tmSFB;
   }
   if (nv) {

@@ -33,36 +33,19 @@ def assert_close(gpu, ref, what=""):
             f"worst at {worst}: gpu={gpu[worst]!r} ref={ref[worst]!r}; first bad {idx.tolist()}")
 
 
-def _sf_offset(r, b, kch):
-    """Byte offset of row r, K-block b in the activation scale layout.
-
-    Rows in blocks of 128, K in chunks of 64 (4 scales).  Inside the 512-byte
-    atom of one (row block, chunk), row r and block j have index
-    a = (r%32)*16 + ((r%128)//32)*4 + j.  Atoms of chunks 2c and 2c+1 form a
-    1 KB pair stored in 128-byte pieces: piece p = bytes [128p, 128p+128) of
-    the even atom, then the same bytes of the odd atom.  ceil(K/256)*4 chunks
-    per row block, stored chunk-fastest.
-    """
-    a = (r % 32) * 16 + ((r % 128) // 32) * 4 + (b % 4)
-    chunk = b // 4
-    return ((r // 128) * kch + (chunk - chunk % 2)) * 512 + (a // 128) * 256 + (chunk % 2) * 128 + a % 128
-
-
 def sf_unswizzle(sf_bytes: np.ndarray, rows: int, K: int) -> np.ndarray:
-    """Undo the activation scale layout -> logical [rows, K/16]."""
+    """Undo the GEMM's scale-factor atom layout -> logical [rows, K/16].
+
+    Atom layout: rows in blocks of 128, K in chunks of 64 (4 scales), 512-byte
+    atoms stored chunk-fastest with ceil(K/256)*4 chunks per row block; inside
+    an atom, row r and K-block j sit at (r%32)*16 + (r//32)*4 + j.
+    """
     kch = ((K + 255) // 256) * 4
     nb = K // 16
     r = np.arange(rows)[:, None]
     b = np.arange(nb)[None, :]
-    return np.asarray(sf_bytes)[_sf_offset(r, b, kch)]
-
-
-def sf_logical_offsets(rows: int, K: int) -> np.ndarray:
-    """Offsets of the real (row < rows, block < K/16) scales, [rows, K/16]."""
-    kch = ((K + 255) // 256) * 4
-    r = np.arange(rows)[:, None]
-    b = np.arange(K // 16)[None, :]
-    return _sf_offset(r, b, kch)
+    off = ((r // 128) * kch + b // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + (b % 4)
+    return np.asarray(sf_bytes)[off]
 
 
 def sf_layout_offsets(rows: int, K: int) -> np.ndarray:
@@ -71,7 +54,7 @@ def sf_layout_offsets(rows: int, K: int) -> np.ndarray:
     mpad = ((rows + 127) // 128) * 128
     r = np.arange(mpad)[:, None]
     b = np.arange(kch * 4)[None, :]
-    return _sf_offset(r, b, kch).ravel()
+    return (((r // 128) * kch + b // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + (b % 4)).ravel()
 
 
 def sample_rows(M: int, n: int, seed: int = 0) -> np.ndarray:
