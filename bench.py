@@ -246,6 +246,51 @@ class Model:
         return n
 
 
+def quant_bytes(layer) -> int:
+    """Algorithmic HBM bytes of one activation quantization of `layer`'s input."""
+    mk = layer.M * layer.K
+    if layer.fmt == "fp8":
+        return mk * 2 + mk + layer.M * 4                # read x, write codes, row scales
+    return mk * 2 + mk * 2 + mk // 2 + mk // 16 + 16    # amax pass, read x, codes, block scales
+
+
+def quant_roofline(model, stream, peaks, peak_src, min_ms=50.0):
+    """The quantize kernel(s) of every layer timed alone (HBM bound), on the
+    same rotating input sets; CUDA events on the launching stream."""
+    import torch
+    out = []
+    for j, layer in enumerate(model.wl.layers):
+        def run(i):
+            layers = model.sets[i % len(model.sets)]
+            x = layers[0]["x"] if j == 0 else layers[j - 1]["out"]
+            d = layers[j]
+            d["lay"].quantize(x, d["codes"], d["scales"], stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                run(i)
+            e0.record(stream)
+            run(0)
+            e1.record(stream)
+        stream.synchronize()
+        n = int(min(2000, max(20, min_ms / max(e0.elapsed_time(e1), 1e-3))))
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(n):
+                run(i)
+            e1.record(stream)
+        stream.synchronize()
+        us = e0.elapsed_time(e1) / n * 1e3
+        gbs = quant_bytes(layer) / (us * 1e-6) / 1e9
+        out.append({"layer": j, "kernel": "quant_fp8_rows" if layer.fmt == "fp8"
+                    else "tensor_amax+quant_nvfp4", "bound": "hbm", "us": round(us, 2),
+                    "bytes": quant_bytes(layer), "achieved": round(gbs, 1),
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(gbs / peaks["hbm_gbs"], 4), "calls": n,
+                    "peak_source": f"{peak_src} copy bandwidth"})
+    return out
+
+
 def cpu_baseline(wl, seconds):
     """Time the oracle (as it stands) on a bounded row sample of the workload's
     first layer; returns TFLOP/s-equivalent and a description."""
@@ -372,6 +417,8 @@ def main_ours(args):
                 "gemm_ms": round(gemm_ms[j], 5), "gemm_launches_timed": len(sampled),
                 "gemm_share": round(sum(gemm_ms) / ms_per_step, 4)}
 
+    quant = quant_roofline(model, stream, peaks, peak_src)
+
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(model, stream, dev, args, world, flops_step)
@@ -398,6 +445,7 @@ def main_ours(args):
                        "l2": f"inputs rotate over {nsets} sets ({per_set / 2**20:.0f} MB each); "
                              "no set is L2-resident when reused"},
             "roofline": roofline,
+            "quant_roofline": quant,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": model.launches_per_step() * args.steps,
