@@ -163,6 +163,36 @@ QL_API ql_status qlinear_forward(qlinear_t h, const void* codes, const void* sca
                           const void* residual, const void* gate, void* out_bf16,
                           void* stream);
 
+/* GEMM + fused epilogue whose result is written as the NEXT NVFP4 layer's
+ * quantized activation instead of bf16 -- the activation quantization fused
+ * into the producing kernel.  Kernel fusion is one of the engine features
+ * listed in wavespeed.ai's "Solucion de WaveSpeed para Acelerar la Generacion
+ * de Imagenes FLUX.1-dev", section "Marco de Inferencia Propietario de
+ * WaveSpeedAI"; the fused-epilogue GEMMs are in algoritmulzilei.ro's FLUX 3
+ * Image Klein page.  Each epilogue value is rounded to bf16 exactly as
+ * qlinear_forward would store it and then quantized to NVFP4 (16-element
+ * blocks along the output columns, E4M3 block scales) with the tensor amax
+ * taken from `amax` instead of from this output: G = amax/2688 and block
+ * scale E4M3(amax_b * 448/amax), the qlinear_quantize_act formulas with the
+ * tensor amax replaced.  Values beyond what `amax` can represent saturate.
+ *   Only NVFP4 layers (QL_ERR_UNSUPPORTED otherwise), Nout % 256 == 0.
+ *   codes, scales, residual, gate : as for qlinear_forward.
+ *   amax       : device fp32 scalar: a calibration value or the amax observed
+ *                on the previous step (read by the kernel, not by the host).
+ *   out_codes  : device [M, Nout/2] bytes; out_scales: device, the block
+ *                scales in the activation layout of a layer with K = Nout,
+ *                followed by the 16-byte tail: fp32 G, then the largest
+ *                |value| of this output as fp32 bits (the observed amax, for
+ *                the next step).  Size both with qlinear_act_bytes of the
+ *                next layer (K = Nout).  The pair is the codes/scales input
+ *                of that layer's qlinear_forward.
+ *   With amax equal to this output's true amax the buffers are byte-identical
+ *   to qlinear_quantize_act of the bf16 output.  No host sync, no allocation. */
+QL_API ql_status qlinear_forward_nvfp4_out(qlinear_t h, const void* codes, const void* scales,
+                                           int64_t M, const void* residual, const void* gate,
+                                           const float* amax, void* out_codes, void* out_scales,
+                                           void* stream);
+
 /* Copy the quantized weights to host memory in logical order (synchronizes).
  *   FP8  : codes_host [N, K] bytes, scales_host fp32 [N], global_scale ignored.
  *   NVFP4: codes_host [N, K/2] bytes, scales_host [N, K/16] E4M3 block-scale

@@ -11,7 +11,8 @@ import numpy as np
 from . import _abi
 from ._abi import (EPILOGUES, FORMATS, QLinearError, make_desc, qlinear_abi_version,  # noqa: F401
                    qlinear_act_bytes, qlinear_check, qlinear_create, qlinear_destroy,
-                   qlinear_export_weights, qlinear_forward, qlinear_out_features,
+                   qlinear_export_weights, qlinear_forward, qlinear_forward_nvfp4_out,
+                   qlinear_out_features,
                    qlinear_quantize_act, qlinear_weight_bytes, status_string)
 
 __all__ = ["QLinear", "make_desc", "QLinearError"]
@@ -61,6 +62,15 @@ class QLinear:
     def forward_codes(self, codes, scales, M, out, residual=None, gate=None, stream=None):
         qlinear_forward(self.h, codes.data_ptr(), scales.data_ptr(), M, _ptr(residual), _ptr(gate),
                         out.data_ptr(), _stream_ptr(stream))
+
+    def forward_nvfp4_out(self, codes, scales, M, amax, out_codes, out_scales, residual=None,
+                          gate=None, stream=None):
+        """GEMM + epilogue written as the next NVFP4 layer's quantized input
+        (codes, scales sized by that layer's act_buffers), against the tensor
+        amax held in the device fp32 tensor `amax`."""
+        qlinear_forward_nvfp4_out(self.h, codes.data_ptr(), scales.data_ptr(), M, _ptr(residual),
+                                  _ptr(gate), amax.data_ptr(), out_codes.data_ptr(),
+                                  out_scales.data_ptr(), _stream_ptr(stream))
 
     def __call__(self, x, residual=None, gate=None, out=None, bufs=None, stream=None):
         import torch

@@ -19,7 +19,7 @@ EPILOGUES = {"bias": 0, "bias_gelu": 1, "swiglu": 2, "bias_gated_residual": 3,
 # every entry point declared in include/qlinear.h
 EXPORTS = ("qlinear_weight_bytes", "qlinear_create", "qlinear_act_bytes", "qlinear_out_features",
            "qlinear_quantize_act", "qlinear_quantize_act_noalloc", "qlinear_forward",
-           "qlinear_export_weights", "qlinear_check", "qlinear_debug_set_fault", "qlinear_destroy",
+           "qlinear_forward_nvfp4_out", "qlinear_export_weights", "qlinear_check", "qlinear_debug_set_fault", "qlinear_destroy",
            "qlinear_status_string", "qlinear_abi_version")
 
 
@@ -57,6 +57,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.qlinear_quantize_act.argtypes = [P, P, i64, P, P, P]
     L.qlinear_quantize_act_noalloc.argtypes = [P, P, i64, P, P, P]
     L.qlinear_forward.argtypes = [P, P, P, i64, P, P, P, P]
+    L.qlinear_forward_nvfp4_out.argtypes = [P, P, P, i64, P, P, P, P, P, P]
     L.qlinear_export_weights.argtypes = [P, P, P, ctypes.POINTER(ctypes.c_float), P]
     L.qlinear_check.argtypes = [P, P]
     L.qlinear_debug_set_fault.argtypes = [P, ctypes.c_int32]
@@ -148,6 +149,15 @@ def qlinear_forward(h, codes_ptr, scales_ptr, M, residual_ptr, gate_ptr, out_ptr
     s = load().qlinear_forward(h, codes_ptr, scales_ptr, M, residual_ptr, gate_ptr, out_ptr, stream)
     if check:
         _ck("qlinear_forward", s)
+    return s
+
+
+def qlinear_forward_nvfp4_out(h, codes_ptr, scales_ptr, M, residual_ptr, gate_ptr, amax_ptr,
+                              out_codes_ptr, out_scales_ptr, stream=0, check=True):
+    s = load().qlinear_forward_nvfp4_out(h, codes_ptr, scales_ptr, M, residual_ptr, gate_ptr,
+                                         amax_ptr, out_codes_ptr, out_scales_ptr, stream)
+    if check:
+        _ck("qlinear_forward_nvfp4_out", s)
     return s
 
 

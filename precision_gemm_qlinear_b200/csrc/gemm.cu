@@ -35,6 +35,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "codec.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -235,7 +236,9 @@ __device__ __forceinline__ void load_f32x32(const float* p, float (&o)[32]) {
   }
 }
 
-template <int FMT, int EPI, int CG>
+// OQ = 1: the epilogue writes NVFP4 codes and block scales for the next
+// layer instead of bf16 (see GemmParams::q_*).
+template <int FMT, int EPI, int CG, int OQ>
 __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_constant__ GemmParams p) {
   using C = Cfg<FMT, CG, EPI>;
   constexpr int BN = C::BN;
@@ -477,6 +480,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
     const uint32_t ovl_l0 = mapa_shared(smem_u32(&sb->ovl_free), 0);
     int local = 0;
     uint32_t nstore = 0;
+    // NVFP4 output: tensor factors from the supplied amax, and the largest
+    // |value| this thread quantizes (for the observed amax)
+    float q_G = 0.f, q_enc = 0.f, qmax = 0.f;
+    if constexpr (OQ) {
+      const float qA = __ldg(p.q_amax);
+      q_G = __fdiv_rn(qA, 2688.f);
+      q_enc = qA > 0.f ? __fdiv_rn(448.f, qA) : 0.f;
+      if (blockIdx.x == 0 && ew == 0 && lane == 0) *p.q_g = q_G;
+    }
     for (int t = unit; t < num_tiles; t += nunits, ++local) {
       int mb, nb;
       tile_coords(t, p, mb, nb);
@@ -602,6 +614,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
           }
         }
         if (!live) continue;
+        if constexpr (OQ) {
+          // two 16-element blocks of the next layer's K: codes for rows < M,
+          // zero scales for the padded rows of the last 128-row block
+          uint2 c0, c1;
+          float a0, a1;
+          const uint32_t sb0 = nvfp4_block(make_uint4(packed[0], packed[1], packed[2], packed[3]),
+                                           make_uint4(packed[4], packed[5], packed[6], packed[7]),
+                                           q_enc, q_G, c0, a0);
+          const uint32_t sb1 =
+              nvfp4_block(make_uint4(packed[8], packed[9], packed[10], packed[11]),
+                          make_uint4(packed[12], packed[13], packed[14], packed[15]), q_enc, q_G,
+                          c1, a1);
+          uint16_t* sfp = reinterpret_cast<uint16_t*>(p.q_sf + sf_offset(m, ocol >> 4, p.q_kchunks));
+          if (row_ok) {
+            *reinterpret_cast<uint4*>(p.q_codes + static_cast<int64_t>(m) * (p.Nout >> 1) +
+                                      (ocol >> 1)) = make_uint4(c0.x, c0.y, c1.x, c1.y);
+            *sfp = static_cast<uint16_t>(sb0 | (sb1 << 8));
+            qmax = fmaxf(qmax, fmaxf(a0, a1));
+          } else if (m < p.q_mpad) {
+            *sfp = 0;
+          }
+          continue;
+        }
         // ---- stage through swizzled shared memory, then one TMA store per warp
         uint8_t* sbuf = staging + (nstore % C::NBUF) * STAGING_BYTES;
         if (lane == 0) bulk_wait_group_read<C::NBUF - 1>();
@@ -622,6 +657,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
       }
     }
     if (lane == 0) bulk_wait_group<0>();
+    if constexpr (OQ) {
+      // |values| >= 0: float bit patterns order like unsigned integers
+      const uint32_t b = __reduce_max_sync(0xffffffffu, __float_as_uint(qmax));
+      if (lane == 0 && b != 0u) atomicMax(p.q_obs, b);
+    }
   }
 
   __syncwarp();
@@ -640,11 +680,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
   }
 }
 
-template <int FMT, int EPI, int CG>
+template <int FMT, int EPI, int CG, int OQ>
 cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t st) {
   using C = Cfg<FMT, CG, EPI>;
   static bool attr_set = false;
-  auto kern = qgemm_kernel<FMT, EPI, CG>;
+  auto kern = qgemm_kernel<FMT, EPI, CG, OQ>;
   if (!attr_set) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -679,12 +719,17 @@ int gemm_tile_n(int fmt, int epi) {
   return epi == EPI_SWIGLU ? Cfg<1, 2, EPI_SWIGLU>::BN : Cfg<1, 2, EPI_BIAS>::BN;
 }
 
-cudaError_t launch_gemm(int fmt, int epi, int cg, const GemmParams& p, int num_sms,
+cudaError_t launch_gemm(int fmt, int epi, int cg, int outq, const GemmParams& p, int num_sms,
                         cudaStream_t st) {
 #define QLB_CASE(F, E)                                                     \
-  if (fmt == F && epi == E) {                                              \
-    return cg == 2 ? launch_one<F, E, 2>(p, num_sms, st)                   \
-                   : launch_one<F, E, 1>(p, num_sms, st);                  \
+  if (fmt == F && epi == E && !outq) {                                     \
+    return cg == 2 ? launch_one<F, E, 2, 0>(p, num_sms, st)                \
+                   : launch_one<F, E, 1, 0>(p, num_sms, st);               \
+  }
+#define QLB_CASE_Q(E)                                                      \
+  if (fmt == 1 && epi == E && outq) {                                      \
+    return cg == 2 ? launch_one<1, E, 2, 1>(p, num_sms, st)                \
+                   : launch_one<1, E, 1, 1>(p, num_sms, st);               \
   }
   QLB_CASE(0, EPI_BIAS)
   QLB_CASE(0, EPI_BIAS_GELU)
@@ -696,7 +741,13 @@ cudaError_t launch_gemm(int fmt, int epi, int cg, const GemmParams& p, int num_s
   QLB_CASE(1, EPI_SWIGLU)
   QLB_CASE(1, EPI_GATED_RES)
   QLB_CASE(1, EPI_SPLIT)
+  QLB_CASE_Q(EPI_BIAS)
+  QLB_CASE_Q(EPI_BIAS_GELU)
+  QLB_CASE_Q(EPI_SWIGLU)
+  QLB_CASE_Q(EPI_GATED_RES)
+  QLB_CASE_Q(EPI_SPLIT)
 #undef QLB_CASE
+#undef QLB_CASE_Q
   return cudaErrorInvalidValue;
 }
 

@@ -120,10 +120,21 @@ struct alignas(64) GemmParams {
   int32_t tiles_m, tiles_n, group_m;
   int32_t sf_kchunks_a, sfb_nstages;
   int32_t fault_mode;     // test hook: 0 = none
+  // NVFP4 output (instead of bf16): the epilogue's bf16 values quantized for a
+  // next layer with K = Nout, against the tensor amax *q_amax supplied by the
+  // caller.  Codes [M, Nout/2]; block scales in the sf_offset layout (padded
+  // rows [M, q_mpad) get zero scales); *q_g = G; *q_obs = max |value| seen.
+  uint8_t* q_codes;
+  uint8_t* q_sf;
+  const float* q_amax;
+  float* q_g;
+  uint32_t* q_obs;
+  int32_t q_kchunks, q_mpad;
 };
 
 // cg = 1: one CTA per 128 x 256 tile; cg = 2: a CTA pair per 256 x 256 tile.
-cudaError_t launch_gemm(int fmt, int epi, int cg, const GemmParams& p, int num_sms,
+// outq = 1: NVFP4 output through the q_* fields (NVFP4 layers only).
+cudaError_t launch_gemm(int fmt, int epi, int cg, int outq, const GemmParams& p, int num_sms,
                         cudaStream_t st);
 // N of the GEMM tile for a format / epilogue (the weight scale layout uses it).
 int gemm_tile_n(int fmt, int epi);

@@ -181,6 +181,102 @@ size_t act_scale_bytes(const qlinear_s* h, int64_t M) {
 
 }  // namespace
 
+namespace {
+
+// NVFP4 output of qlinear_forward_nvfp4_out.
+struct QOut {
+  void* codes;
+  void* scales;
+  const float* amax;
+};
+
+ql_status forward_impl(qlinear_t h, const void* codes, const void* scales, int64_t M,
+                       const void* residual, const void* gate, void* out_bf16, const QOut* q,
+                       void* stream) {
+  if (!h || M < 0 || M > 0x7FFFFFFF) return QL_ERR_INVALID_ARG;
+  if (M == 0) return QL_OK;
+  if (!codes || !scales || (!q && !out_bf16)) return QL_ERR_INVALID_ARG;
+  const bool gated = h->d.epi == QL_EPI_BIAS_GATED_RESIDUAL;
+  if (gated && (!residual || !gate)) return QL_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(scales) || (!q && !aligned16(out_bf16)))
+    return QL_ERR_ALIGNMENT;
+  if (gated && (!aligned16(residual) || !aligned16(gate))) return QL_ERR_ALIGNMENT;
+  if (h->Nout % 8 != 0) return QL_ERR_ALIGNMENT;
+  const bool nv = h->d.fmt == QL_NVFP4;
+  if (q) {
+    if (!nv || h->Nout % 256 != 0) return QL_ERR_UNSUPPORTED;
+    if (!q->codes || !q->scales || !q->amax) return QL_ERR_INVALID_ARG;
+    if (!aligned16(q->codes) || !aligned16(q->scales) ||
+        (reinterpret_cast<uintptr_t>(q->amax) & 3) != 0)
+      return QL_ERR_ALIGNMENT;
+  }
+
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  const uint64_t kbytes = nv ? h->K / 2 : h->K;
+  // one CTA per 128-row tile for a single M tile, else CTA pairs on 256 rows
+  const int cg = h->d.variant == 1 ? 1 : (h->d.variant == 2 ? 2 : (M > 128 ? 2 : 1));
+  if (!make_tmap(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, kbytes, M, kbytes, 128, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return QL_ERR_CUDA;
+  if (!q && !make_tmap(&p.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out_bf16, h->Nout, M,
+                       h->Nout * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return QL_ERR_CUDA;
+  p.tmB = cg == 2 ? h->tmB2 : h->tmB1;
+  if (nv && cg == 2) {
+    if (!make_sf_tmap(&p.tmSFA, scales, sf_bytes(M, h->K), 1)) return QL_ERR_CUDA;
+    p.tmSFB = h->tmSFB;
+  }
+  if (nv) {
+    p.sfa = static_cast<const uint8_t*>(scales);
+    p.ga = reinterpret_cast<const float*>(p.sfa + sf_bytes(M, h->K));
+    p.sfb = h->wsf;
+    p.gw = h->wG;
+  } else {
+    p.sa = static_cast<const float*>(scales);
+    p.sw = h->wscale;
+  }
+  p.bias = h->bias;
+  p.residual = static_cast<const __nv_bfloat16*>(residual);
+  p.gate = static_cast<const __nv_bfloat16*>(gate);
+  p.out = static_cast<__nv_bfloat16*>(out_bf16);
+  p.err = h->err;
+  p.M = static_cast<int32_t>(M);
+  p.N = static_cast<int32_t>(h->N);
+  p.Nout = static_cast<int32_t>(h->Nout);
+  p.split_col = static_cast<int32_t>(h->d.split_col);
+  p.k_blocks = static_cast<int32_t>((kbytes + 127) / 128);
+  p.tiles_m = static_cast<int32_t>((M + 128 * cg - 1) / (128 * cg));
+  p.tiles_n = static_cast<int32_t>((h->N + h->bn - 1) / h->bn);
+  p.group_m = 8;
+  p.sf_kchunks_a = static_cast<int32_t>(sf_kchunks(h->K));
+  p.sfb_nstages = static_cast<int32_t>(sfb_stages(h->K));
+  p.fault_mode = h->fault_mode;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (q) {
+    uint8_t* sf = static_cast<uint8_t*>(q->scales);
+    p.q_codes = static_cast<uint8_t*>(q->codes);
+    p.q_sf = sf;
+    p.q_amax = q->amax;
+    p.q_g = reinterpret_cast<float*>(sf + sf_bytes(M, h->Nout));
+    p.q_obs = reinterpret_cast<uint32_t*>(p.q_g + 1);
+    p.q_kchunks = static_cast<int32_t>(sf_kchunks(h->Nout));
+    p.q_mpad = static_cast<int32_t>((M + 127) / 128 * 128);
+    if (cudaMemsetAsync(p.q_obs, 0, 4, st) != cudaSuccess) {
+      cudaGetLastError();
+      return QL_ERR_CUDA;
+    }
+  }
+  cudaError_t e = launch_gemm(h->d.fmt, h->d.epi, cg, q ? 1 : 0, p, h->num_sms, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int32_t qlinear_abi_version(void) { return kAbiVersion; }
@@ -328,63 +424,14 @@ ql_status qlinear_quantize_act_noalloc(qlinear_t h, const void* x_bf16, int64_t 
 
 ql_status qlinear_forward(qlinear_t h, const void* codes, const void* scales, int64_t M,
                           const void* residual, const void* gate, void* out_bf16, void* stream) {
-  if (!h || M < 0 || M > 0x7FFFFFFF) return QL_ERR_INVALID_ARG;
-  if (M == 0) return QL_OK;
-  if (!codes || !scales || !out_bf16) return QL_ERR_INVALID_ARG;
-  const bool gated = h->d.epi == QL_EPI_BIAS_GATED_RESIDUAL;
-  if (gated && (!residual || !gate)) return QL_ERR_INVALID_ARG;
-  if (!aligned16(codes) || !aligned16(scales) || !aligned16(out_bf16)) return QL_ERR_ALIGNMENT;
-  if (gated && (!aligned16(residual) || !aligned16(gate))) return QL_ERR_ALIGNMENT;
-  if (h->Nout % 8 != 0) return QL_ERR_ALIGNMENT;
+  return forward_impl(h, codes, scales, M, residual, gate, out_bf16, nullptr, stream);
+}
 
-  GemmParams p;
-  std::memset(&p, 0, sizeof(p));
-  const bool nv = h->d.fmt == QL_NVFP4;
-  const uint64_t kbytes = nv ? h->K / 2 : h->K;
-  // one CTA per 128-row tile for a single M tile, else CTA pairs on 256 rows
-  const int cg = h->d.variant == 1 ? 1 : (h->d.variant == 2 ? 2 : (M > 128 ? 2 : 1));
-  if (!make_tmap(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, kbytes, M, kbytes, 128, 128,
-                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap(&p.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out_bf16, h->Nout, M, h->Nout * 2, 32,
-                 32, CU_TENSOR_MAP_SWIZZLE_64B))
-    return QL_ERR_CUDA;
-  p.tmB = cg == 2 ? h->tmB2 : h->tmB1;
-  if (nv && cg == 2) {
-    if (!make_sf_tmap(&p.tmSFA, scales, sf_bytes(M, h->K), 1)) return QL_ERR_CUDA;
-    p.tmSFB = h->tmSFB;
-  }
-  if (nv) {
-    p.sfa = static_cast<const uint8_t*>(scales);
-    p.ga = reinterpret_cast<const float*>(p.sfa + sf_bytes(M, h->K));
-    p.sfb = h->wsf;
-    p.gw = h->wG;
-  } else {
-    p.sa = static_cast<const float*>(scales);
-    p.sw = h->wscale;
-  }
-  p.bias = h->bias;
-  p.residual = static_cast<const __nv_bfloat16*>(residual);
-  p.gate = static_cast<const __nv_bfloat16*>(gate);
-  p.out = static_cast<__nv_bfloat16*>(out_bf16);
-  p.err = h->err;
-  p.M = static_cast<int32_t>(M);
-  p.N = static_cast<int32_t>(h->N);
-  p.Nout = static_cast<int32_t>(h->Nout);
-  p.split_col = static_cast<int32_t>(h->d.split_col);
-  p.k_blocks = static_cast<int32_t>((kbytes + 127) / 128);
-  p.tiles_m = static_cast<int32_t>((M + 128 * cg - 1) / (128 * cg));
-  p.tiles_n = static_cast<int32_t>((h->N + h->bn - 1) / h->bn);
-  p.group_m = 8;
-  p.sf_kchunks_a = static_cast<int32_t>(sf_kchunks(h->K));
-  p.sfb_nstages = static_cast<int32_t>(sfb_stages(h->K));
-  p.fault_mode = h->fault_mode;
-  cudaError_t e =
-      launch_gemm(h->d.fmt, h->d.epi, cg, p, h->num_sms, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return QL_ERR_CUDA;
-  }
-  return QL_OK;
+ql_status qlinear_forward_nvfp4_out(qlinear_t h, const void* codes, const void* scales, int64_t M,
+                                    const void* residual, const void* gate, const float* amax,
+                                    void* out_codes, void* out_scales, void* stream) {
+  const QOut q{out_codes, out_scales, amax};
+  return forward_impl(h, codes, scales, M, residual, gate, nullptr, &q, stream);
 }
 
 ql_status qlinear_export_weights(qlinear_t h, void* codes_host, void* scales_host,

@@ -17,40 +17,13 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "codec.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace qlb {
 
 namespace {
-
-__device__ __forceinline__ float absmax8(const uint4& v) {
-  // |bf16| max over 8 values, done on the bit patterns' float images
-  float m = fmaxf(fabsf(bf16lo(v.x)), fabsf(bf16hi(v.x)));
-  m = fmaxf(m, fmaxf(fabsf(bf16lo(v.y)), fabsf(bf16hi(v.y))));
-  m = fmaxf(m, fmaxf(fabsf(bf16lo(v.z)), fabsf(bf16hi(v.z))));
-  m = fmaxf(m, fmaxf(fabsf(bf16lo(v.w)), fabsf(bf16hi(v.w))));
-  return m;
-}
-
-__device__ __forceinline__ uint32_t e4m3_pair(uint32_t w, float inv) {
-  // bf16x2 word -> 2 E4M3 codes (element 0 in the low byte)
-  return cvt_e4m3x2(__fmul_rn(bf16hi(w), inv), __fmul_rn(bf16lo(w), inv));
-}
-
-__device__ __forceinline__ uint2 e4m3_8(const uint4& v, float inv) {
-  uint2 r;
-  r.x = e4m3_pair(v.x, inv) | (e4m3_pair(v.y, inv) << 16);
-  r.y = e4m3_pair(v.z, inv) | (e4m3_pair(v.w, inv) << 16);
-  return r;
-}
-
-__device__ __forceinline__ uint32_t e2m1_4(const uint2& w, float inv) {
-  // 4 bf16 -> 4 E2M1 codes packed in 16 bits (element 0 in the low nibble)
-  uint32_t b0 = cvt_e2m1x2(__fmul_rn(bf16hi(w.x), inv), __fmul_rn(bf16lo(w.x), inv));
-  uint32_t b1 = cvt_e2m1x2(__fmul_rn(bf16hi(w.y), inv), __fmul_rn(bf16lo(w.y), inv));
-  return b0 | (b1 << 8);
-}
 
 __device__ __forceinline__ uint4 ld_nc(const uint4* p) {
   uint4 v;
@@ -184,14 +157,9 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
       const int64_t b = g * 4 + i;
       if (b < nb) {
         const uint4* xp = reinterpret_cast<const uint4*>(xr + b * 16);
-        const uint4 v0 = ld_nc(xp), v1 = ld_nc(xp + 1);
-        const float amb = fmaxf(absmax8(v0), absmax8(v1));
-        const uint32_t sb = cvt_e4m3x2(0.f, __fmul_rn(amb, enc)) & 0xFF;
-        const float den = __fmul_rn(e4m3_to_f32(sb), G);
-        const float inv = den > 0.f ? __fdiv_rn(1.f, den) : 0.f;
         uint2 out;
-        out.x = e2m1_4(make_uint2(v0.x, v0.y), inv) | (e2m1_4(make_uint2(v0.z, v0.w), inv) << 16);
-        out.y = e2m1_4(make_uint2(v1.x, v1.y), inv) | (e2m1_4(make_uint2(v1.z, v1.w), inv) << 16);
+        float amb;
+        const uint32_t sb = nvfp4_block(ld_nc(xp), ld_nc(xp + 1), enc, G, out, amb);
         *reinterpret_cast<uint2*>(q + row * (K >> 1) + b * 8) = out;
         word |= sb << (8 * i);
       }

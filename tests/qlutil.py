@@ -48,6 +48,14 @@ def sf_unswizzle(sf_bytes: np.ndarray, rows: int, K: int) -> np.ndarray:
     return np.asarray(sf_bytes)[off]
 
 
+def sf_logical_offsets(rows: int, K: int) -> np.ndarray:
+    """Offsets of the real scales (row < rows, block < K/16), shape [rows, K/16]."""
+    kch = ((K + 255) // 256) * 4
+    r = np.arange(rows)[:, None]
+    b = np.arange(K // 16)[None, :]
+    return ((r // 128) * kch + b // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + (b % 4)
+
+
 def sf_layout_offsets(rows: int, K: int) -> np.ndarray:
     """Every (row, block) offset of the padded scale layout, for the bijection test."""
     kch = ((K + 255) // 256) * 4
