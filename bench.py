@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--sets", type=int, default=0, help="input rotation sets (0 = auto)")
+    ap.add_argument("--fuse-quant", action="store_true",
+                    help="NVFP4 -> NVFP4 layer boundaries: the producing GEMM writes the next "
+                         "layer's quantized input (previous step's observed amax)")
     ap.add_argument("--gemm-event-every", type=int, default=8,
                     help="record per-GEMM CUDA events on every n-th timed step")
     ap.add_argument("--tokens", type=int, default=0,
@@ -193,9 +196,15 @@ def to_dev(a, dev):
 
 
 class Model:
-    """The workload's layers with NSETS rotated copies of inputs and weights."""
+    """The workload's layers with NSETS rotated copies of inputs and weights.
 
-    def __init__(self, wl, dev, seed, nsets):
+    fuse=True: at every NVFP4 -> NVFP4 layer boundary (Nout % 256 == 0) the
+    producing GEMM writes the next layer's quantized input itself
+    (qlinear_forward_nvfp4_out), against the tensor amax the same boundary
+    observed on the previous step (another input set); a calibration pass of
+    the unfused path provides the first values."""
+
+    def __init__(self, wl, dev, seed, nsets, fuse=False):
         import torch
         import precision_gemm_qlinear_b200 as ql
         self.wl, self.dev = wl, dev
@@ -221,28 +230,64 @@ class Model:
                 layers.append(d)
             self.sets.append(layers)
         self.host0 = host0
+        L = wl.layers
+        self.fused = [False] + [
+            fuse and L[j - 1].fmt == "nvfp4" and L[j].fmt == "nvfp4" and
+            (L[j - 1].N // 2 if L[j - 1].epi == "swiglu" else L[j - 1].N) % 256 == 0
+            for j in range(1, len(L))]
+        if fuse and not any(self.fused):
+            raise ValueError(f"{wl.name}: no NVFP4 -> NVFP4 boundary to fuse")
         torch.cuda.synchronize()
+        if any(self.fused):
+            for s in range(nsets):   # calibration: the unfused path fills every observed amax
+                self.run_layers(self.sets[s], self.sets[s][0]["x"], None, unfused=True)
+            torch.cuda.synchronize()
 
-    def step(self, s, stream, gemm_events=None):
-        """Enqueue one pass of the path over input set s."""
-        layers = self.sets[s % len(self.sets)]
-        x = layers[0]["x"]
+    def amax_of(self, layers, j):
+        """Device fp32 view of the observed tensor amax stored in the tail of
+        layer j's activation scales of one input set."""
+        import torch
+        layer = self.wl.layers[j]
+        nsf = ((layer.M + 127) // 128) * ((layer.K + 255) // 256) * 4 * 512
+        return layers[j]["scales"][nsf + 4:nsf + 8].view(torch.float32)
+
+    def run_layers(self, layers, x, stream, gemm_events=None, amax_from=None, unfused=False):
+        """quantize + GEMM + epilogue of every layer over one input set."""
         for i, d in enumerate(layers):
             lay = d["lay"]
-            lay.quantize(x, d["codes"], d["scales"], stream)
+            fused_in = self.fused[i] and not unfused
+            fused_out = i + 1 < len(layers) and self.fused[i + 1] and not unfused
+            if not fused_in:
+                lay.quantize(x, d["codes"], d["scales"], stream)
+            M = self.wl.layers[i].M
             if gemm_events is not None:
                 gemm_events[i][0].record(stream)
-            lay.forward_codes(d["codes"], d["scales"], x.shape[0], d["out"], d.get("residual"),
-                              d.get("gate"), stream)
+            if fused_out:
+                nd = layers[i + 1]
+                lay.forward_nvfp4_out(d["codes"], d["scales"], M, self.amax_of(amax_from, i + 1),
+                                      nd["codes"], nd["scales"], d.get("residual"), d.get("gate"),
+                                      stream)
+            else:
+                lay.forward_codes(d["codes"], d["scales"], M, d["out"], d.get("residual"),
+                                  d.get("gate"), stream)
             if gemm_events is not None:
                 gemm_events[i][1].record(stream)
             x = d["out"]
         return x
 
+    def step(self, s, stream, gemm_events=None):
+        """Enqueue one pass of the path over input set s."""
+        n = len(self.sets)
+        layers = self.sets[s % n]
+        return self.run_layers(layers, layers[0]["x"], stream, gemm_events,
+                               amax_from=self.sets[(s - 1) % n])
+
     def launches_per_step(self):
         n = 0
-        for layer in self.wl.layers:
-            n += 2 if layer.fmt == "fp8" else 3
+        for j, layer in enumerate(self.wl.layers):
+            if not self.fused[j]:
+                n += 1 if layer.fmt == "fp8" else 2   # the quantize kernels
+            n += 1                                     # the GEMM
         return n
 
 
@@ -260,6 +305,8 @@ def quant_roofline(model, stream, peaks, peak_src, min_ms=50.0):
     import torch
     out = []
     for j, layer in enumerate(model.wl.layers):
+        if model.fused[j]:
+            continue  # quantized by the previous layer's epilogue, no kernel of its own
         def run(i):
             layers = model.sets[i % len(model.sets)]
             x = layers[0]["x"] if j == 0 else layers[j - 1]["out"]
@@ -351,7 +398,7 @@ def main_ours(args):
         per_set += layer.M * layer.K * 2 + layer.N * kb + layer.M * (
             layer.N // 2 if layer.epi == "swiglu" else layer.N) * 2
     nsets = args.sets or max(2, int(np.ceil(2 * L2_BYTES / per_set)) + 1)
-    model = Model(wl, dev, seed=rank_seed(rank), nsets=nsets)
+    model = Model(wl, dev, seed=rank_seed(rank), nsets=nsets, fuse=args.fuse_quant)
     stream = torch.cuda.Stream(device=dev)
     flops_step = float(wl.flops)
 
@@ -442,6 +489,7 @@ def main_ours(args):
             "config": {"workload": wl.name, "desc": wl.note,
                        "layers": [dict(fmt=l.fmt, M=l.M, K=l.K, N=l.N, epi=l.epi) for l in wl.layers],
                        "global_tokens": wl.layers[0].M * world, "parallelism": f"replicas{world}",
+                       "fused_quant": [j for j, f in enumerate(model.fused) if f],
                        "l2": f"inputs rotate over {nsets} sets ({per_set / 2**20:.0f} MB each); "
                              "no set is L2-resident when reused"},
             "roofline": roofline,
@@ -473,13 +521,7 @@ def run_e2e(model, stream, dev, args, world, flops_step):
     with torch.cuda.stream(stream):
         def one():
             x_dev.copy_(x_host, non_blocking=True)
-            x = x_dev
-            for d in model.sets[0]:
-                lay = d["lay"]
-                lay.quantize(x, d["codes"], d["scales"], stream)
-                lay.forward_codes(d["codes"], d["scales"], x.shape[0], d["out"],
-                                  d.get("residual"), d.get("gate"), stream)
-                x = d["out"]
+            x = model.run_layers(model.sets[0], x_dev, stream, amax_from=model.sets[1 % len(model.sets)])
             out_host.copy_(x, non_blocking=True)
         for _ in range(3):
             one()

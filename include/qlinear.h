@@ -108,6 +108,26 @@ QL_API ql_status qlinear_weight_bytes(const ql_desc* desc, size_t* bytes);
 QL_API ql_status qlinear_create(const ql_desc* desc, const void* w_bf16, const void* bias_bf16,
                          void* weight_ws, size_t ws_bytes, void* stream, qlinear_t* out);
 
+/* Build a layer from weights that are already quantized -- a pre-quantized
+ * checkpoint (algoritmulzilei.ro, "Accelerarea generarii de imagini cu FLUX 3
+ * Image Klein pe GPU-urile Blackwell": the runtime loads BFL's pre-quantized
+ * NVFP4 DiT checkpoints; paragraph after Table 1).  The weights come in the
+ * logical order that qlinear_export_weights returns, so export followed by
+ * this call rebuilds an identical layer:
+ *   FP8  : codes [N, K] E4M3 bytes; scales fp32 [N] (s_w per output channel).
+ *   NVFP4: codes [N, K/2] bytes (element 2j in the low nibble); scales
+ *          [N, K/16] E4M3 block-scale bytes; global_scale = G (host value,
+ *          finite and >= 0; ignored for FP8).
+ *   codes, scales : device, 16-byte aligned; read by kernels enqueued on
+ *                   `stream` (keep them alive until the stream passes them).
+ *   Everything else as for qlinear_create (same workspace size and layout;
+ *   SwiGLU rows are interleaved by the library, the caller passes gate rows
+ *   0..N/2-1 then up rows). */
+QL_API ql_status qlinear_create_prequantized(const ql_desc* desc, const void* codes,
+                                             const void* scales, float global_scale,
+                                             const void* bias_bf16, void* weight_ws,
+                                             size_t ws_bytes, void* stream, qlinear_t* out);
+
 /* Sizes of the activation code and scale buffers for M tokens.
  *   FP8  : codes [M, K] bytes; scales fp32 [M] (rounded up to 16 bytes).
  *   NVFP4: codes [M, K/2] bytes (two codes per byte, low nibble first);
@@ -162,6 +182,16 @@ QL_API ql_status qlinear_quantize_act_noalloc(qlinear_t h, const void* x_bf16, i
 QL_API ql_status qlinear_forward(qlinear_t h, const void* codes, const void* scales, int64_t M,
                           const void* residual, const void* gate, void* out_bf16,
                           void* stream);
+
+/* qlinear_forward for QL_EPI_BIAS_GATED_RESIDUAL layers whose adaLN gate
+ * differs between groups of tokens, as when the conditional and the
+ * unconditional passes of classifier-free guidance are batched into one M:
+ * gate is device [ceil(M / rows_per_gate), Nout] bf16 and token m uses gate
+ * row m / rows_per_gate (residual + gate[m / rows_per_gate] * (y + b)).
+ * rows_per_gate >= 1; other epilogues return QL_ERR_INVALID_ARG. */
+QL_API ql_status qlinear_forward_gate_rows(qlinear_t h, const void* codes, const void* scales,
+                                           int64_t M, const void* residual, const void* gate,
+                                           int64_t rows_per_gate, void* out_bf16, void* stream);
 
 /* GEMM + fused epilogue whose result is written as the NEXT NVFP4 layer's
  * quantized activation instead of bf16 -- the activation quantization fused

@@ -10,7 +10,8 @@ import numpy as np
 
 from . import _abi
 from ._abi import (EPILOGUES, FORMATS, QLinearError, make_desc, qlinear_abi_version,  # noqa: F401
-                   qlinear_act_bytes, qlinear_check, qlinear_create, qlinear_destroy,
+                   qlinear_act_bytes, qlinear_check, qlinear_create, qlinear_create_prequantized,
+                   qlinear_destroy, qlinear_forward_gate_rows,
                    qlinear_export_weights, qlinear_forward, qlinear_forward_nvfp4_out,
                    qlinear_out_features,
                    qlinear_quantize_act, qlinear_weight_bytes, status_string)
@@ -48,6 +49,26 @@ class QLinear:
                                 _stream_ptr(stream))
         self.Nout = qlinear_out_features(self.h)
 
+    @classmethod
+    def from_quantized(cls, fmt, epi, codes, scales, global_scale=0.0, bias=None, split_col=0,
+                       variant=0, stream=None):
+        """A layer from pre-quantized weights in the order export_weights
+        returns: codes uint8 CUDA [N, K] (FP8) or [N, K/2] (NVFP4); scales
+        fp32 [N] (FP8) or uint8 [N, K/16] E4M3 block scales (NVFP4); G."""
+        import torch
+        self = cls.__new__(cls)
+        N = int(codes.shape[0])
+        K = int(codes.shape[1]) * (2 if fmt == "nvfp4" else 1)
+        self.fmt, self.epi, self.N, self.K = fmt, epi, N, K
+        self.desc = make_desc(fmt, epi, N, K, split_col, variant)
+        nbytes = qlinear_weight_bytes(self.desc)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=codes.device)
+        self.h = qlinear_create_prequantized(self.desc, codes.data_ptr(), scales.data_ptr(),
+                                             float(global_scale), _ptr(bias), self.ws.data_ptr(),
+                                             nbytes, _stream_ptr(stream))
+        self.Nout = qlinear_out_features(self.h)
+        return self
+
     def act_buffers(self, M, device="cuda"):
         import torch
         cb, sb = qlinear_act_bytes(self.h, M)
@@ -62,6 +83,13 @@ class QLinear:
     def forward_codes(self, codes, scales, M, out, residual=None, gate=None, stream=None):
         qlinear_forward(self.h, codes.data_ptr(), scales.data_ptr(), M, _ptr(residual), _ptr(gate),
                         out.data_ptr(), _stream_ptr(stream))
+
+    def forward_codes_gate_rows(self, codes, scales, M, out, residual, gate, rows_per_gate,
+                                stream=None):
+        """Gated-residual forward with gate [ceil(M / rows_per_gate), Nout]."""
+        qlinear_forward_gate_rows(self.h, codes.data_ptr(), scales.data_ptr(), M,
+                                  residual.data_ptr(), gate.data_ptr(), rows_per_gate,
+                                  out.data_ptr(), _stream_ptr(stream))
 
     def forward_nvfp4_out(self, codes, scales, M, amax, out_codes, out_scales, residual=None,
                           gate=None, stream=None):

@@ -17,9 +17,10 @@ EPILOGUES = {"bias": 0, "bias_gelu": 1, "swiglu": 2, "bias_gated_residual": 3,
              "split_bias_gelu": 4}
 
 # every entry point declared in include/qlinear.h
-EXPORTS = ("qlinear_weight_bytes", "qlinear_create", "qlinear_act_bytes", "qlinear_out_features",
+EXPORTS = ("qlinear_weight_bytes", "qlinear_create", "qlinear_create_prequantized",
+           "qlinear_act_bytes", "qlinear_out_features",
            "qlinear_quantize_act", "qlinear_quantize_act_noalloc", "qlinear_forward",
-           "qlinear_forward_nvfp4_out", "qlinear_export_weights", "qlinear_check", "qlinear_debug_set_fault", "qlinear_destroy",
+           "qlinear_forward_gate_rows", "qlinear_forward_nvfp4_out", "qlinear_export_weights", "qlinear_check", "qlinear_debug_set_fault", "qlinear_destroy",
            "qlinear_status_string", "qlinear_abi_version")
 
 
@@ -58,6 +59,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.qlinear_quantize_act_noalloc.argtypes = [P, P, i64, P, P, P]
     L.qlinear_forward.argtypes = [P, P, P, i64, P, P, P, P]
     L.qlinear_forward_nvfp4_out.argtypes = [P, P, P, i64, P, P, P, P, P, P]
+    L.qlinear_forward_gate_rows.argtypes = [P, P, P, i64, P, P, i64, P, P]
+    L.qlinear_create_prequantized.argtypes = [D, P, P, ctypes.c_float, P, P, sz, P,
+                                              ctypes.POINTER(P)]
     L.qlinear_export_weights.argtypes = [P, P, P, ctypes.POINTER(ctypes.c_float), P]
     L.qlinear_check.argtypes = [P, P]
     L.qlinear_debug_set_fault.argtypes = [P, ctypes.c_int32]
@@ -111,6 +115,18 @@ def qlinear_create(desc: ql_desc, w_ptr, bias_ptr, ws_ptr, ws_bytes, stream=0, c
     return s, h.value
 
 
+def qlinear_create_prequantized(desc: ql_desc, codes_ptr, scales_ptr, global_scale, bias_ptr,
+                                ws_ptr, ws_bytes, stream=0, check=True):
+    h = ctypes.c_void_p(0)
+    s = load().qlinear_create_prequantized(ctypes.byref(desc), codes_ptr, scales_ptr,
+                                           ctypes.c_float(global_scale), bias_ptr, ws_ptr, ws_bytes,
+                                           stream, ctypes.byref(h))
+    if check:
+        _ck("qlinear_create_prequantized", s)
+        return h.value
+    return s, h.value
+
+
 def qlinear_act_bytes(h, M, check=True):
     c, sc = ctypes.c_size_t(0), ctypes.c_size_t(0)
     s = load().qlinear_act_bytes(h, M, ctypes.byref(c), ctypes.byref(sc))
@@ -149,6 +165,15 @@ def qlinear_forward(h, codes_ptr, scales_ptr, M, residual_ptr, gate_ptr, out_ptr
     s = load().qlinear_forward(h, codes_ptr, scales_ptr, M, residual_ptr, gate_ptr, out_ptr, stream)
     if check:
         _ck("qlinear_forward", s)
+    return s
+
+
+def qlinear_forward_gate_rows(h, codes_ptr, scales_ptr, M, residual_ptr, gate_ptr, rows_per_gate,
+                              out_ptr, stream=0, check=True):
+    s = load().qlinear_forward_gate_rows(h, codes_ptr, scales_ptr, M, residual_ptr, gate_ptr,
+                                         rows_per_gate, out_ptr, stream)
+    if check:
+        _ck("qlinear_forward_gate_rows", s)
     return s
 
 

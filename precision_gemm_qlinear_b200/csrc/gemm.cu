@@ -539,7 +539,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
             if constexpr (!C::NV) load_f32x32(p.sw + ncol + 128, sw_b);
           }
           if constexpr (EPI == EPI_GATED_RES) {
-            load_bf16x32_packed(p.gate + ocol, gate_a);
+            // per-batch gates (CFG-batched tokens): row m uses gate row m / gate_rows
+            const __nv_bfloat16* gp = p.gate + ocol;
+            if (p.gate_rows > 0)
+              gp += static_cast<int64_t>((row_ok ? m : p.M - 1) / p.gate_rows) * p.Nout;
+            load_bf16x32_packed(gp, gate_a);
             if (row_ok) {
               load_bf16x32_packed(p.residual + static_cast<int64_t>(m) * p.Nout + ocol, res_a);
             } else {

@@ -83,6 +83,13 @@ inline cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStr
 
 cudaError_t launch_quant_fp8_rows(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
                                   float* s, RowMap map, int num_sms, cudaStream_t st);
+// Pre-quantized weights in logical order (fmt 0: codes [N, K], fp32 row scales
+// [N]; fmt 1: codes [N, K/2], block scales [N, K/16]) -> the GEMM's layout
+// (rows permuted by map; NVFP4 scales replicated as the quantizer writes them,
+// into a zeroed region).
+cudaError_t launch_import_weights(int fmt, const void* codes, const void* scales, int64_t N,
+                                  int64_t K, int64_t bn, uint8_t* wcodes, void* wscales, RowMap map,
+                                  cudaStream_t st);
 cudaError_t launch_tensor_amax(const void* x, int64_t n_elems, uint32_t* amax_bits, int num_sms,
                                cudaStream_t st);
 // sf_layout: 0 = activation (A operand) atoms [sf_offset], 1 = weight (B
@@ -120,6 +127,7 @@ struct alignas(64) GemmParams {
   int32_t tiles_m, tiles_n, group_m;
   int32_t sf_kchunks_a, sfb_nstages;
   int32_t fault_mode;     // test hook: 0 = none
+  int32_t gate_rows;      // gated residual: 0 = one gate [Nout]; else gate [M/gate_rows, Nout]
   // NVFP4 output (instead of bf16): the epilogue's bf16 values quantized for a
   // next layer with K = Nout, against the tensor amax *q_amax supplied by the
   // caller.  Codes [M, Nout/2]; block scales in the sf_offset layout (padded

@@ -191,13 +191,15 @@ struct QOut {
 };
 
 ql_status forward_impl(qlinear_t h, const void* codes, const void* scales, int64_t M,
-                       const void* residual, const void* gate, void* out_bf16, const QOut* q,
-                       void* stream) {
+                       const void* residual, const void* gate, int64_t gate_rows, void* out_bf16,
+                       const QOut* q, void* stream) {
   if (!h || M < 0 || M > 0x7FFFFFFF) return QL_ERR_INVALID_ARG;
   if (M == 0) return QL_OK;
   if (!codes || !scales || (!q && !out_bf16)) return QL_ERR_INVALID_ARG;
   const bool gated = h->d.epi == QL_EPI_BIAS_GATED_RESIDUAL;
   if (gated && (!residual || !gate)) return QL_ERR_INVALID_ARG;
+  if (gate_rows < 0 || gate_rows > 0x7FFFFFFF || (gate_rows > 0 && !gated))
+    return QL_ERR_INVALID_ARG;
   if (!aligned16(codes) || !aligned16(scales) || (!q && !aligned16(out_bf16)))
     return QL_ERR_ALIGNMENT;
   if (gated && (!aligned16(residual) || !aligned16(gate))) return QL_ERR_ALIGNMENT;
@@ -252,6 +254,7 @@ ql_status forward_impl(qlinear_t h, const void* codes, const void* scales, int64
   p.sf_kchunks_a = static_cast<int32_t>(sf_kchunks(h->K));
   p.sfb_nstages = static_cast<int32_t>(sfb_stages(h->K));
   p.fault_mode = h->fault_mode;
+  p.gate_rows = static_cast<int32_t>(gate_rows);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (q) {
     uint8_t* sf = static_cast<uint8_t*>(q->scales);
@@ -272,6 +275,77 @@ ql_status forward_impl(qlinear_t h, const void* codes, const void* scales, int64
     cudaGetLastError();
     return QL_ERR_CUDA;
   }
+  return QL_OK;
+}
+
+}  // namespace
+
+namespace {
+
+// Checks shared by both ways of creating a layer, then the handle with its
+// workspace pointers (nothing launched yet).
+ql_status begin_create(const ql_desc* desc, const void* bias_bf16, void* weight_ws,
+                       size_t ws_bytes, qlinear_s** hp) {
+  ql_status s = check_desc(desc);
+  if (s != QL_OK) return s;
+  if (!weight_ws) return QL_ERR_INVALID_ARG;
+  if ((bias_bf16 && !aligned16(bias_bf16)) || (reinterpret_cast<uintptr_t>(weight_ws) & 255) != 0)
+    return QL_ERR_ALIGNMENT;
+  const WsLayout L = ws_layout(*desc);
+  if (ws_bytes < L.total) return QL_ERR_INVALID_ARG;
+  DevInfo di;
+  if ((s = current_device(&di)) != QL_OK) return s;
+  if (di.major != 10) return QL_ERR_UNSUPPORTED;
+
+  qlinear_s* h = new (std::nothrow) qlinear_s();
+  if (!h) return QL_ERR_INVALID_ARG;
+  h->d = *desc;
+  h->N = desc->N;
+  h->K = desc->K;
+  h->Nout = desc->epi == QL_EPI_SWIGLU ? desc->N / 2 : desc->N;
+  h->device = di.device;
+  h->num_sms = di.num_sms;
+  h->ws = static_cast<uint8_t*>(weight_ws);
+  h->ws_bytes = ws_bytes;
+  h->err = reinterpret_cast<uint32_t*>(h->ws + L.err);
+  h->wcodes = h->ws + L.codes;
+  h->bias = reinterpret_cast<__nv_bfloat16*>(h->ws + L.bias);
+  h->map.nout = h->Nout;
+  h->map.mode = desc->epi == QL_EPI_SWIGLU ? 1 : 0;
+  h->bn = gemm_tile_n(desc->fmt, desc->epi);
+  if (desc->fmt == QL_FP8_E4M3) {
+    h->wscale = reinterpret_cast<float*>(h->ws + L.scales);
+  } else {
+    h->wsf = h->ws + L.scales;
+    h->wG = reinterpret_cast<float*>(h->wsf + sfb_bytes(h->N, h->K, h->bn));
+    h->wamax = reinterpret_cast<uint32_t*>(h->wG + 1);
+  }
+  *hp = h;
+  return QL_OK;
+}
+
+// The bias and the tensor maps of the weight operand; frees the handle when
+// anything failed (including the weight kernels' launch status `e`).
+ql_status finish_create(qlinear_s* h, cudaError_t e, const void* bias_bf16, cudaStream_t st,
+                        qlinear_t* out) {
+  if (e == cudaSuccess) e = launch_permute_bias(bias_bf16, h->bias, h->N, h->map, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return QL_ERR_CUDA;
+  }
+  const uint64_t kbytes = h->d.fmt == QL_NVFP4 ? h->K / 2 : h->K;
+  bool ok = make_tmap(&h->tmB1, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, 128,
+                      h->bn, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            make_tmap(&h->tmB2, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, 128,
+                      h->bn / 2, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (ok && h->d.fmt == QL_NVFP4)
+    ok = make_sf_tmap(&h->tmSFB, h->wsf, sfb_bytes(h->N, h->K, h->bn), 8);
+  if (!ok) {
+    delete h;
+    return QL_ERR_CUDA;
+  }
+  *out = h;
   return QL_OK;
 }
 
@@ -305,72 +379,53 @@ ql_status qlinear_create(const ql_desc* desc, const void* w_bf16, const void* bi
                          void* weight_ws, size_t ws_bytes, void* stream, qlinear_t* out) {
   if (!out) return QL_ERR_INVALID_ARG;
   *out = nullptr;
-  ql_status s = check_desc(desc);
+  if (!w_bf16) return QL_ERR_INVALID_ARG;
+  if (!aligned16(w_bf16)) return QL_ERR_ALIGNMENT;
+  qlinear_s* h = nullptr;
+  ql_status s = begin_create(desc, bias_bf16, weight_ws, ws_bytes, &h);
   if (s != QL_OK) return s;
-  if (!w_bf16 || !weight_ws) return QL_ERR_INVALID_ARG;
-  if (!aligned16(w_bf16) || (bias_bf16 && !aligned16(bias_bf16)) ||
-      (reinterpret_cast<uintptr_t>(weight_ws) & 255) != 0)
-    return QL_ERR_ALIGNMENT;
-  const WsLayout L = ws_layout(*desc);
-  if (ws_bytes < L.total) return QL_ERR_INVALID_ARG;
-  DevInfo di;
-  if ((s = current_device(&di)) != QL_OK) return s;
-  if (di.major != 10) return QL_ERR_UNSUPPORTED;
-
-  qlinear_s* h = new (std::nothrow) qlinear_s();
-  if (!h) return QL_ERR_INVALID_ARG;
-  h->d = *desc;
-  h->N = desc->N;
-  h->K = desc->K;
-  h->Nout = desc->epi == QL_EPI_SWIGLU ? desc->N / 2 : desc->N;
-  h->device = di.device;
-  h->num_sms = di.num_sms;
-  h->ws = static_cast<uint8_t*>(weight_ws);
-  h->ws_bytes = ws_bytes;
-  h->err = reinterpret_cast<uint32_t*>(h->ws + L.err);
-  h->wcodes = h->ws + L.codes;
-  h->bias = reinterpret_cast<__nv_bfloat16*>(h->ws + L.bias);
-  h->map.nout = h->Nout;
-  h->map.mode = desc->epi == QL_EPI_SWIGLU ? 1 : 0;
-  h->bn = gemm_tile_n(desc->fmt, desc->epi);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-
   cudaError_t e = cudaMemsetAsync(h->ws, 0, 1024, st);
   if (e == cudaSuccess && desc->fmt == QL_FP8_E4M3) {
-    h->wscale = reinterpret_cast<float*>(h->ws + L.scales);
     e = launch_quant_fp8_rows(w_bf16, h->N, h->K, h->K, h->wcodes, h->wscale, h->map, h->num_sms,
                               st);
   } else if (e == cudaSuccess) {
-    h->wsf = h->ws + L.scales;
-    h->wG = reinterpret_cast<float*>(h->wsf + sfb_bytes(h->N, h->K, h->bn));
-    h->wamax = reinterpret_cast<uint32_t*>(h->wG + 1);
     // unused scale words (rows past N, word 7 of a 224-row tile) stay zero
     e = cudaMemsetAsync(h->wsf, 0, sfb_bytes(h->N, h->K, h->bn) + 16, st);
     if (e == cudaSuccess) e = launch_tensor_amax(w_bf16, h->N * h->K, h->wamax, h->num_sms, st);
     if (e == cudaSuccess)
       e = launch_quant_nvfp4(w_bf16, h->N, h->K, h->K, h->wcodes, h->wsf, 1, h->bn, h->wamax, h->wG,
-                             h->map,
-                             st);
+                             h->map, st);
   }
-  if (e == cudaSuccess) e = launch_permute_bias(bias_bf16, h->bias, h->N, h->map, st);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    delete h;
-    return QL_ERR_CUDA;
+  return finish_create(h, e, bias_bf16, st, out);
+}
+
+ql_status qlinear_create_prequantized(const ql_desc* desc, const void* codes, const void* scales,
+                                      float global_scale, const void* bias_bf16, void* weight_ws,
+                                      size_t ws_bytes, void* stream, qlinear_t* out) {
+  if (!out) return QL_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!codes || !scales) return QL_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(scales)) return QL_ERR_ALIGNMENT;
+  if (desc && desc->fmt == QL_NVFP4 && !(global_scale >= 0.f && global_scale <= 3.4e38f))
+    return QL_ERR_INVALID_ARG;  // negative, infinite or NaN
+  qlinear_s* h = nullptr;
+  ql_status s = begin_create(desc, bias_bf16, weight_ws, ws_bytes, &h);
+  if (s != QL_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(h->ws, 0, 1024, st);
+  if (e == cudaSuccess && desc->fmt == QL_NVFP4) {
+    e = cudaMemsetAsync(h->wsf, 0, sfb_bytes(h->N, h->K, h->bn) + 16, st);
+    // G from a host value: the copy is staged before the call returns
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(h->wG, &global_scale, sizeof(float), cudaMemcpyHostToDevice, st);
   }
-  const uint64_t kbytes = desc->fmt == QL_NVFP4 ? h->K / 2 : h->K;
-  bool ok = make_tmap(&h->tmB1, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, 128,
-                      h->bn, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            make_tmap(&h->tmB2, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, 128,
-                      h->bn / 2, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (ok && desc->fmt == QL_NVFP4)
-    ok = make_sf_tmap(&h->tmSFB, h->wsf, sfb_bytes(h->N, h->K, h->bn), 8);
-  if (!ok) {
-    delete h;
-    return QL_ERR_CUDA;
-  }
-  *out = h;
-  return QL_OK;
+  if (e == cudaSuccess)
+    e = launch_import_weights(desc->fmt == QL_NVFP4 ? 1 : 0, codes, scales, h->N, h->K, h->bn,
+                              h->wcodes, desc->fmt == QL_NVFP4 ? static_cast<void*>(h->wsf)
+                                                               : static_cast<void*>(h->wscale),
+                              h->map, st);
+  return finish_create(h, e, bias_bf16, st, out);
 }
 
 ql_status qlinear_act_bytes(qlinear_t h, int64_t M, size_t* code_bytes, size_t* scale_bytes) {
@@ -424,14 +479,22 @@ ql_status qlinear_quantize_act_noalloc(qlinear_t h, const void* x_bf16, int64_t 
 
 ql_status qlinear_forward(qlinear_t h, const void* codes, const void* scales, int64_t M,
                           const void* residual, const void* gate, void* out_bf16, void* stream) {
-  return forward_impl(h, codes, scales, M, residual, gate, out_bf16, nullptr, stream);
+  return forward_impl(h, codes, scales, M, residual, gate, 0, out_bf16, nullptr, stream);
+}
+
+ql_status qlinear_forward_gate_rows(qlinear_t h, const void* codes, const void* scales, int64_t M,
+                                    const void* residual, const void* gate, int64_t rows_per_gate,
+                                    void* out_bf16, void* stream) {
+  if (rows_per_gate < 1) return QL_ERR_INVALID_ARG;
+  return forward_impl(h, codes, scales, M, residual, gate, rows_per_gate, out_bf16, nullptr,
+                      stream);
 }
 
 ql_status qlinear_forward_nvfp4_out(qlinear_t h, const void* codes, const void* scales, int64_t M,
                                     const void* residual, const void* gate, const float* amax,
                                     void* out_codes, void* out_scales, void* stream) {
   const QOut q{out_codes, out_scales, amax};
-  return forward_impl(h, codes, scales, M, residual, gate, nullptr, &q, stream);
+  return forward_impl(h, codes, scales, M, residual, gate, 0, nullptr, &q, stream);
 }
 
 ql_status qlinear_export_weights(qlinear_t h, void* codes_host, void* scales_host,

@@ -174,6 +174,45 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
   }
 }
 
+// ---------------------------------------------------- pre-quantized import
+
+// Row n of the GEMM's weight operand is logical row map(n) (SwiGLU
+// interleave); rows of `row_bytes` bytes, 16 bytes per thread.
+__global__ void import_rows_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                   int64_t N, int64_t row_vecs, RowMap map) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= N * row_vecs) return;
+  const int64_t n = i / row_vecs, v = i - n * row_vecs;
+  dst[i] = src[map(n) * row_vecs + v];
+}
+
+__global__ void import_row_scales_kernel(const float* __restrict__ src, float* __restrict__ dst,
+                                         int64_t N, RowMap map) {
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (n < N) dst[n] = src[map(n)];
+}
+
+// Logical NVFP4 block scales [N, K/16] -> the replicated weight layout, one
+// thread per (row, group of 4 blocks), the same words the weight quantizer
+// writes (blocks past K/16 are 0).
+__global__ void import_block_scales_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ sf,
+                                           int64_t N, int64_t K, int64_t bn, RowMap map) {
+  const int64_t nks = sfb_stages(K);
+  const int64_t ngp = nks * 4;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= N * ngp) return;
+  const int64_t row = idx / ngp, g = idx - row * ngp;
+  const int64_t nb = K >> 4;
+  const uint8_t* sr = src + map(row) * nb;
+  uint32_t word = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (g * 4 + i < nb) word |= static_cast<uint32_t>(sr[g * 4 + i]) << (8 * i);
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4)
+    *reinterpret_cast<uint32_t*>(sf + sfb_word_offset(row, g >> 2, g & 3, q4, nks, bn)) = word;
+}
+
 __global__ void permute_bias_kernel(const __nv_bfloat16* __restrict__ src,
                                     __nv_bfloat16* __restrict__ dst, int64_t N, RowMap map) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -208,6 +247,24 @@ cudaError_t launch_quant_fp8_rows(const void* x, int64_t M, int64_t K, int64_t l
   }
   cudaLaunchConfig_t c = pdl_config(grid_for(1), 256, 0, st, at, 0);
   return cudaLaunchKernelEx(&c, quant_fp8_rows_kernel<256, VPL>, xb, M, K, ldx, q, s, map);
+}
+
+cudaError_t launch_import_weights(int fmt, const void* codes, const void* scales, int64_t N,
+                                  int64_t K, int64_t bn, uint8_t* wcodes, void* wscales, RowMap map,
+                                  cudaStream_t st) {
+  const int64_t row_vecs = (fmt == 1 ? K / 2 : K) / 16;
+  const int64_t nv = N * row_vecs;
+  import_rows_kernel<<<static_cast<unsigned>((nv + 255) / 256), 256, 0, st>>>(
+      static_cast<const uint4*>(codes), reinterpret_cast<uint4*>(wcodes), N, row_vecs, map);
+  if (fmt == 0) {
+    import_row_scales_kernel<<<static_cast<unsigned>((N + 255) / 256), 256, 0, st>>>(
+        static_cast<const float*>(scales), static_cast<float*>(wscales), N, map);
+  } else {
+    const int64_t nt = N * sfb_stages(K) * 4;
+    import_block_scales_kernel<<<static_cast<unsigned>((nt + 255) / 256), 256, 0, st>>>(
+        static_cast<const uint8_t*>(scales), static_cast<uint8_t*>(wscales), N, K, bn, map);
+  }
+  return cudaGetLastError();
 }
 
 cudaError_t launch_tensor_amax(const void* x, int64_t n_elems, uint32_t* amax_bits, int num_sms,

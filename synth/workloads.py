@@ -67,6 +67,11 @@ WORKLOADS = {
     "flux2k_swiglu_nvfp4": Workload("flux2k_swiglu_nvfp4", (
         Layer("nvfp4", 16896, 3072, 16384, "swiglu", _T4, bias_std=None),
     ), "NVFP4 2048^2 MLP up-projection with SwiGLU, 16896x3072x(2x8192)"),
+    "flux2k_mlp_nvfp4": Workload("flux2k_mlp_nvfp4", (
+        Layer("nvfp4", 16896, 3072, 16384, "swiglu", _T4, bias_std=None),
+        Layer("nvfp4", 16896, 8192, 3072, "bias_gated_residual", _N01, chained=True),
+    ), "NVFP4 2048^2 MLP pair: up 16896x3072x(2x8192) SwiGLU, down 16896x8192x3072 "
+       "residual + gate*(xW+b)"),
     "cfg_linear1_fp8": Workload("cfg_linear1_fp8", (
         Layer("fp8", 33792, 3072, 21504, "split_bias_gelu", _T3_OUT20, split_col=9216),
     ), "CFG-batched parallel-block linear1, FP8, 33792x3072x21504, split bias/GELU"),
