@@ -129,48 +129,67 @@ __global__ void __launch_bounds__(256) tensor_amax_kernel(const uint4* __restric
 
 // ------------------------------------------------------- NVFP4 block quant
 
-// One thread per 64 elements (4 blocks of 16) of a row.  Threads cover the
-// padded grid [ceil(M/128)*128 rows, ceil(K/256)*4 groups] so that every
-// padding scale is written as zero.
+// One warp per row of the padded grid [mpad rows, nks * 256 columns]: in each
+// step a lane takes one 16-byte vector (8 elements), so a warp reads 512
+// contiguous bytes per load; the two lanes of a 16-element block exchange
+// their maxima with one shuffle, and the 4 scale bytes of a 64-element group
+// (lanes 8i, 8i+2, 8i+4, 8i+6) are gathered into one word.  U steps of loads
+// are issued before any is used.  Rows are taken in reverse order so that the
+// first ones processed are the tensor's tail, which the amax pass read last
+// and which is still in L2.  Padding rows and K groups get zero scales.
+template <int U>
 __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
     const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K, int64_t ldx,
     uint8_t* __restrict__ q, uint8_t* __restrict__ sf, int sf_layout, int64_t bn, int64_t nks,
-    int64_t mpad,
-    const uint32_t* __restrict__ amax_bits, float* g_out, RowMap map) {
-  const int64_t ngp = nks * 4;  // padded 64-element groups per row
-  const int64_t nb = K >> 4;
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t row = idx / ngp;
-  const int64_t g = idx - row * ngp;
+    int64_t mpad, const uint32_t* __restrict__ amax_bits, float* g_out, RowMap map) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   grid_dep_wait();  // the tensor amax of the previous kernel
   grid_dep_launch_dependents();
-  if (row >= mpad) return;
+  if (w >= mpad) return;  // warp-uniform
+  const int64_t row = mpad - 1 - w;
   const float A = __uint_as_float(*amax_bits);
   const float G = __fdiv_rn(A, 2688.f);
   const float enc = A > 0.f ? __fdiv_rn(448.f, A) : 0.f;
-  if (idx == 0 && g_out != nullptr) *g_out = G;
-  uint32_t word = 0;  // the 4 block-scale codes of this group, block 4g in the low byte
-  if (row < M) {
-    const __nv_bfloat16* xr = x + map(row) * ldx;
+  if (w == 0 && lane == 0 && g_out != nullptr) *g_out = G;
+  const bool live = row < M;
+  const int64_t nvec = K >> 3;  // 16-byte vectors of a row
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (live ? map(row) : 0) * ldx);
+  uint32_t* qr = reinterpret_cast<uint32_t*>(q + (live ? row : 0) * (K >> 1));
+  for (int64_t s0 = 0; s0 < nks; s0 += U) {
+    uint4 v[U];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int64_t b = g * 4 + i;
-      if (b < nb) {
-        const uint4* xp = reinterpret_cast<const uint4*>(xr + b * 16);
-        uint2 out;
-        float amb;
-        const uint32_t sb = nvfp4_block(ld_nc(xp), ld_nc(xp + 1), enc, G, out, amb);
-        *reinterpret_cast<uint2*>(q + row * (K >> 1) + b * 8) = out;
-        word |= sb << (8 * i);
+    for (int u = 0; u < U; ++u) {
+      const int64_t vi = (s0 + u) * 32 + lane;
+      v[u] = (live && s0 + u < nks && vi < nvec) ? ld_nc(xr + vi) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (s0 + u >= nks) break;  // warp-uniform
+      const int64_t vi = (s0 + u) * 32 + lane;
+      float amb = absmax8(v[u]);
+      amb = fmaxf(amb, __shfl_xor_sync(0xffffffffu, amb, 1));  // the block's other half
+      const uint32_t sb = cvt_e4m3x2(0.f, __fmul_rn(amb, enc)) & 0xFF;
+      const float den = __fmul_rn(e4m3_to_f32(sb), G);
+      const float inv = den > 0.f ? __fdiv_rn(1.f, den) : 0.f;
+      if (live && vi < nvec)
+        qr[vi] = e2m1_4(make_uint2(v[u].x, v[u].y), inv) | (e2m1_4(make_uint2(v[u].z, v[u].w), inv) << 16);
+      const uint32_t b1 = __shfl_down_sync(0xffffffffu, sb, 2);
+      const uint32_t b2 = __shfl_down_sync(0xffffffffu, sb, 4);
+      const uint32_t b3 = __shfl_down_sync(0xffffffffu, sb, 6);
+      if ((lane & 7) == 0) {
+        const uint32_t word = sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        const int64_t g = (s0 + u) * 4 + (lane >> 3);  // 64-element group of the row
+        if (sf_layout == 0) {
+          *reinterpret_cast<uint32_t*>(sf + sf_offset(row, g * 4, nks * 4)) = word;
+        } else {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            *reinterpret_cast<uint32_t*>(sf + sfb_word_offset(row, g >> 2, g & 3, q4, nks, bn)) =
+                word;
+        }
       }
     }
-  }
-  if (sf_layout == 0) {
-    *reinterpret_cast<uint32_t*>(sf + sf_offset(row, g * 4, nks * 4)) = word;
-  } else {
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4)
-      *reinterpret_cast<uint32_t*>(sf + sfb_word_offset(row, g >> 2, g & 3, q4, nks, bn)) = word;
   }
 }
 
@@ -285,12 +304,11 @@ cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx,
   // weights (layout 1) pad rows to the N tile, activations to 128
   const int64_t mpad = sf_layout == 1 ? ((M + bn - 1) / bn) * bn : ((M + 127) / 128) * 128;
   const int64_t nks = sfb_stages(K);  // == sf_kchunks(K) / 4
-  const int64_t total = mpad * nks * 4;
-  if (total <= 0) return cudaSuccess;
-  const int64_t blocks = (total + 255) / 256;
+  if (mpad <= 0 || nks <= 0) return cudaSuccess;
+  const int64_t blocks = (mpad + 7) / 8;  // 8 warps (rows) per CTA
   cudaLaunchAttribute at[1];
   cudaLaunchConfig_t c = pdl_config(static_cast<unsigned>(blocks), 256, 0, st, at, 0);
-  return cudaLaunchKernelEx(&c, quant_nvfp4_kernel, static_cast<const __nv_bfloat16*>(x), M, K,
+  return cudaLaunchKernelEx(&c, quant_nvfp4_kernel<4>, static_cast<const __nv_bfloat16*>(x), M, K,
                             ldx, q, sf, sf_layout, bn, nks, mpad, amax_bits, g_out, map);
 }
 
