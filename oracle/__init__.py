@@ -45,6 +45,7 @@ def lib():
         L.or_gemm_nvfp4.argtypes = [P, P, ctypes.c_float, P, P, ctypes.c_float, i64, i64, P,
                                     i64, P]
         L.or_epilogue.argtypes = [ctypes.c_int, P, i64, i64, P, P, P, P, i64, P]
+        L.or_qkv_norm_rope.argtypes = [P, i64, i64, i64, P, P, P, P, P, P, ctypes.c_double, P]
         L.or_gelu_tanh.restype = ctypes.c_double
         L.or_gelu_tanh.argtypes = [ctypes.c_double]
         L.or_silu.restype = ctypes.c_double
@@ -171,6 +172,25 @@ def epilogue(kind: str, y, bias=None, residual=None, gate=None, rows=None, split
     out = np.empty((nrows, Nout), np.float64)
     lib().or_epilogue(k, _p(y), nrows, N, _p(bias), _p(residual), _p(rows), _p(gate),
                       int(split_col), _p(out))
+    return out
+
+
+def qkv_norm_rope(y, bias, qw, kw, rope_cos, rope_sin, D=128, eps=1e-6, rows=None):
+    """QKV epilogue with per-head RMS normalization of q and k and rotary
+    embedding of their pairs (C: or_qkv_norm_rope).  y [nrows, 3*H*D]
+    (binary64, e.g. the GEMM result of the listed rows); bias bf16 [N] or None;
+    qw, kw bf16 [D]; rope_cos, rope_sin fp32 [tokens, D/2] indexed by rows.
+    Returns the pre-bf16 reference [nrows, N]."""
+    y = _c(y, np.float64)
+    nrows, N = y.shape
+    assert N % (3 * D) == 0 and D % 2 == 0
+    rows = np.arange(nrows, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    bias = None if bias is None else _c(bias, np.uint16)
+    qw, kw = _c(qw, np.uint16), _c(kw, np.uint16)
+    rc, rs = _c(rope_cos, np.float32), _c(rope_sin, np.float32)
+    out = np.empty((nrows, N), np.float64)
+    lib().or_qkv_norm_rope(_p(y), nrows, N, int(D), _p(bias), _p(qw), _p(kw), _p(rc), _p(rs),
+                           _p(rows), ctypes.c_double(eps), _p(out))
     return out
 
 

@@ -345,6 +345,47 @@ void or_epilogue(int kind, const double* y, int64_t nrows, int64_t N, const uint
   }
 }
 
+/* QKV projection epilogue with query/key normalization and rotary position
+ * embedding.  The fused QKV GEMM of algoritmulzilei.ro's "Accelerarea
+ * generarii de imagini cu FLUX 3 Image Klein pe GPU-urile Blackwell" applies
+ * "query/key normalization and rotary position embeddings"; the page gives no
+ * formula, so the plain readings are taken:
+ *   y [nrows, N], N = 3 * H * D: columns [0, N/3) are q, [N/3, 2N/3) are k,
+ *   [2N/3, N) are v, each H heads of D consecutive columns.
+ *   Every column: v = y + b (bias bf16 [N], NULL = 0).
+ *   q and k heads: RMS normalization over the head's D values,
+ *     u_d = v_d / sqrt(mean_d(v_d^2) + eps) * w_d   (w = qw or kw, bf16 [D]),
+ *   then rotary embedding of the pairs (u_{2i}, u_{2i+1}), i < D/2:
+ *     (a, b) -> (a cos - b sin, a sin + b cos),
+ *   cos = rc[rows[r] * D/2 + i], sin = rs[rows[r] * D/2 + i] (fp32 tables,
+ *   one angle per token and pair; the positions are the caller's).
+ * out [nrows, N] binary64, before bf16 rounding. */
+void or_qkv_norm_rope(const double* y, int64_t nrows, int64_t N, int64_t D,
+                      const uint16_t* bias, const uint16_t* qw, const uint16_t* kw,
+                      const float* rc, const float* rs, const int64_t* rows, double eps,
+                      double* out) {
+  const int64_t qk = 2 * (N / 3);
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < nrows; ++r) {
+    for (int64_t n = 0; n < N; ++n)
+      out[r * N + n] = y[r * N + n] + (bias ? (double)bf16_to_f32(bias[n]) : 0.0);
+    for (int64_t h0 = 0; h0 < qk; h0 += D) {
+      double* u = out + r * N + h0;
+      const uint16_t* w = (h0 < N / 3) ? qw : kw;
+      double ss = 0.0;
+      for (int64_t d = 0; d < D; ++d) ss += u[d] * u[d];
+      const double scale = 1.0 / sqrt(ss / (double)D + eps);
+      for (int64_t d = 0; d < D; ++d) u[d] = u[d] * scale * (double)bf16_to_f32(w[d]);
+      for (int64_t i = 0; i < D / 2; ++i) {
+        const double c = rc[rows[r] * (D / 2) + i], sn = rs[rows[r] * (D / 2) + i];
+        const double a = u[2 * i], b = u[2 * i + 1];
+        u[2 * i] = a * c - b * sn;
+        u[2 * i + 1] = a * sn + b * c;
+      }
+    }
+  }
+}
+
 /* Number of OpenMP threads the oracle runs with (1 without OpenMP). */
 int or_num_threads(void) {
 #ifdef _OPENMP
