@@ -227,6 +227,10 @@ class Model:
                 if layer.epi == "bias_gated_residual":
                     d["gate"] = to_dev(inp["gate"], dev)
                     d["residual"] = to_dev(inp["residual"], dev)
+                if layer.epi == "qkv_norm_rope":
+                    lay.set_qk_norm(to_dev(inp["q_norm"], dev), to_dev(inp["k_norm"], dev))
+                    d["rope_cos"] = torch.from_numpy(inp["rope_cos"]).to(dev)
+                    d["rope_sin"] = torch.from_numpy(inp["rope_sin"]).to(dev)
                 layers.append(d)
             self.sets.append(layers)
         self.host0 = host0
@@ -267,6 +271,9 @@ class Model:
                 lay.forward_nvfp4_out(d["codes"], d["scales"], M, self.amax_of(amax_from, i + 1),
                                       nd["codes"], nd["scales"], d.get("residual"), d.get("gate"),
                                       stream)
+            elif "rope_cos" in d:
+                lay.forward_rope(d["codes"], d["scales"], M, d["rope_cos"], d["rope_sin"],
+                                 d["out"], stream)
             else:
                 lay.forward_codes(d["codes"], d["scales"], M, d["out"], d.get("residual"),
                                   d.get("gate"), stream)

@@ -70,7 +70,11 @@ typedef enum {
                                       N = 2*Nout, weight rows [0,Nout) = gate,
                                       [Nout,N) = up                                */
   QL_EPI_BIAS_GATED_RESIDUAL = 3,  /* out = residual + gate[n] * (y + b)  (adaLN)  */
-  QL_EPI_SPLIT_BIAS_GELU = 4       /* n < split_col: y + b ; else gelu_tanh(y + b) */
+  QL_EPI_SPLIT_BIAS_GELU = 4,      /* n < split_col: y + b ; else gelu_tanh(y + b) */
+  QL_EPI_QKV_NORM_ROPE = 5         /* QKV projection: columns [0,N/3) q, [N/3,2N/3) k,
+                                      [2N/3,N) v, heads of 128; v: y + b; q, k heads:
+                                      RMS-normalized (weights, eps: qlinear_set_qk_norm)
+                                      then pairs (2i,2i+1) rotated (qlinear_forward_rope) */
 } ql_epilogue;
 
 /* Layer description.  y = dequant(codes_x) @ dequant(codes_w)^T, shape [M, N]. */
@@ -85,8 +89,8 @@ typedef struct {
 } ql_desc;
 
 /* Shape rules (QL_ERR_INVALID_ARG otherwise):
- *   FP8  : K % 16 == 0, N % 32 == 0;  NVFP4: K % 32 == 0, N % 256 == 0;
- *   SwiGLU: N % 256 == 0;  1 <= K <= 2^24, 1 <= N <= 2^24, 0 <= M <= 2^31-1;
+ *   FP8  : K % 16 == 0, N % 32 == 0;  NVFP4: K % 32 == 0, N % 32 == 0;
+ *   SwiGLU: N % 256 == 0;  QKV with norm + RoPE: N % 768 == 0;  1 <= K <= 2^24, 1 <= N <= 2^24, 0 <= M <= 2^31-1;
  *   split_col % 32 == 0 for the split epilogue.
  */
 
@@ -182,6 +186,27 @@ QL_API ql_status qlinear_quantize_act_noalloc(qlinear_t h, const void* x_bf16, i
 QL_API ql_status qlinear_forward(qlinear_t h, const void* codes, const void* scales, int64_t M,
                           const void* residual, const void* gate, void* out_bf16,
                           void* stream);
+
+/* QL_EPI_QKV_NORM_ROPE: the QKV projection with query/key normalization and
+ * rotary position embedding in the epilogue (algoritmulzilei.ro, "Accelerarea
+ * generarii de imagini cu FLUX 3 Image Klein pe GPU-urile Blackwell": fused
+ * GEMMs include QKV projections with query/key normalization and rotary
+ * position embeddings; the page gives no formula).  Readings: every column
+ * gets y + b; each 128-column q or k head is RMS-normalized,
+ * u = v / sqrt(mean(v^2) + eps) * w  (w = the q or k weight vector), then
+ * each pair (u[2i], u[2i+1]) is rotated: (a c - b s, a s + b c) with
+ * c = rope_cos[m][i], s = rope_sin[m][i] for token m (fp32 tables
+ * [M][64], device, 16-byte aligned; the positions behind the angles are the
+ * caller's).  v heads are stored as y + b.
+ *   qlinear_set_qk_norm: q and k weight vectors (device bf16 [128] each) and
+ *   eps (finite, >= 0); until it is called the weights are 1 and eps 1e-6.
+ *   qlinear_forward_rope: the forward call of such a layer (qlinear_forward
+ *   returns QL_ERR_INVALID_ARG for it: the tables are required). */
+QL_API ql_status qlinear_set_qk_norm(qlinear_t h, const void* q_weight_bf16,
+                                     const void* k_weight_bf16, float eps, void* stream);
+QL_API ql_status qlinear_forward_rope(qlinear_t h, const void* codes, const void* scales,
+                                      int64_t M, const float* rope_cos, const float* rope_sin,
+                                      void* out_bf16, void* stream);
 
 /* qlinear_forward for QL_EPI_BIAS_GATED_RESIDUAL layers whose adaLN gate
  * differs between groups of tokens, as when the conditional and the

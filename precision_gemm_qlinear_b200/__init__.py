@@ -11,7 +11,8 @@ import numpy as np
 from . import _abi
 from ._abi import (EPILOGUES, FORMATS, QLinearError, make_desc, qlinear_abi_version,  # noqa: F401
                    qlinear_act_bytes, qlinear_check, qlinear_create, qlinear_create_prequantized,
-                   qlinear_destroy, qlinear_forward_gate_rows,
+                   qlinear_destroy, qlinear_forward_gate_rows, qlinear_forward_rope,
+                   qlinear_set_qk_norm,
                    qlinear_export_weights, qlinear_forward, qlinear_forward_nvfp4_out,
                    qlinear_out_features,
                    qlinear_quantize_act, qlinear_weight_bytes, status_string)
@@ -90,6 +91,16 @@ class QLinear:
         qlinear_forward_gate_rows(self.h, codes.data_ptr(), scales.data_ptr(), M,
                                   residual.data_ptr(), gate.data_ptr(), rows_per_gate,
                                   out.data_ptr(), _stream_ptr(stream))
+
+    def set_qk_norm(self, q_weight, k_weight, eps=1e-6, stream=None):
+        """QKV layers: bf16 CUDA norm weights [128] for q and k heads, and eps."""
+        qlinear_set_qk_norm(self.h, q_weight.data_ptr(), k_weight.data_ptr(), eps,
+                            _stream_ptr(stream))
+
+    def forward_rope(self, codes, scales, M, rope_cos, rope_sin, out, stream=None):
+        """QKV layers: forward with fp32 CUDA rotary tables [M, 64] (cos, sin)."""
+        qlinear_forward_rope(self.h, codes.data_ptr(), scales.data_ptr(), M, rope_cos.data_ptr(),
+                             rope_sin.data_ptr(), out.data_ptr(), _stream_ptr(stream))
 
     def forward_nvfp4_out(self, codes, scales, M, amax, out_codes, out_scales, residual=None,
                           gate=None, stream=None):

@@ -14,13 +14,14 @@ QL_OK, QL_ERR_INVALID_ARG, QL_ERR_ALIGNMENT, QL_ERR_UNSUPPORTED, QL_ERR_CUDA, QL
 QL_FP8_E4M3, QL_NVFP4 = 0, 1
 FORMATS = {"fp8": QL_FP8_E4M3, "nvfp4": QL_NVFP4}
 EPILOGUES = {"bias": 0, "bias_gelu": 1, "swiglu": 2, "bias_gated_residual": 3,
-             "split_bias_gelu": 4}
+             "split_bias_gelu": 4, "qkv_norm_rope": 5}
 
 # every entry point declared in include/qlinear.h
 EXPORTS = ("qlinear_weight_bytes", "qlinear_create", "qlinear_create_prequantized",
            "qlinear_act_bytes", "qlinear_out_features",
            "qlinear_quantize_act", "qlinear_quantize_act_noalloc", "qlinear_forward",
-           "qlinear_forward_gate_rows", "qlinear_forward_nvfp4_out", "qlinear_export_weights", "qlinear_check", "qlinear_debug_set_fault", "qlinear_destroy",
+           "qlinear_forward_gate_rows", "qlinear_forward_nvfp4_out", "qlinear_forward_rope",
+           "qlinear_set_qk_norm", "qlinear_export_weights", "qlinear_check", "qlinear_debug_set_fault", "qlinear_destroy",
            "qlinear_status_string", "qlinear_abi_version")
 
 
@@ -60,6 +61,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.qlinear_forward.argtypes = [P, P, P, i64, P, P, P, P]
     L.qlinear_forward_nvfp4_out.argtypes = [P, P, P, i64, P, P, P, P, P, P]
     L.qlinear_forward_gate_rows.argtypes = [P, P, P, i64, P, P, i64, P, P]
+    L.qlinear_forward_rope.argtypes = [P, P, P, i64, P, P, P, P]
+    L.qlinear_set_qk_norm.argtypes = [P, P, P, ctypes.c_float, P]
     L.qlinear_create_prequantized.argtypes = [D, P, P, ctypes.c_float, P, P, sz, P,
                                               ctypes.POINTER(P)]
     L.qlinear_export_weights.argtypes = [P, P, P, ctypes.POINTER(ctypes.c_float), P]
@@ -174,6 +177,21 @@ def qlinear_forward_gate_rows(h, codes_ptr, scales_ptr, M, residual_ptr, gate_pt
                                          rows_per_gate, out_ptr, stream)
     if check:
         _ck("qlinear_forward_gate_rows", s)
+    return s
+
+
+def qlinear_forward_rope(h, codes_ptr, scales_ptr, M, cos_ptr, sin_ptr, out_ptr, stream=0,
+                         check=True):
+    s = load().qlinear_forward_rope(h, codes_ptr, scales_ptr, M, cos_ptr, sin_ptr, out_ptr, stream)
+    if check:
+        _ck("qlinear_forward_rope", s)
+    return s
+
+
+def qlinear_set_qk_norm(h, q_ptr, k_ptr, eps=1e-6, stream=0, check=True):
+    s = load().qlinear_set_qk_norm(h, q_ptr, k_ptr, ctypes.c_float(eps), stream)
+    if check:
+        _ck("qlinear_set_qk_norm", s)
     return s
 
 

@@ -74,7 +74,7 @@ struct Cfg {
   // Tile N: 256, except NVFP4 without SwiGLU, where 224 lets two fp32
   // accumulators (2 x 224 TMEM columns) and the 48 scale-factor columns fit
   // in the 512 columns side by side.
-  static constexpr int BN = (NV && EPI != EPI_SWIGLU) ? 224 : 256;
+  static constexpr int BN = (NV && EPI != EPI_SWIGLU && EPI != EPI_QKV) ? 224 : 256;
   static constexpr int B_BYTES = (BN / CG) * BK_BYTES;  // this CTA's rows of B
   static constexpr int SFA_BYTES = NV ? 2048 : 0;       // 4 atoms (one per MMA K step)
   static constexpr int SFB_BYTES = NV ? 16384 : 0;      // 4 replicated 4 KB chunks (all 256 B rows)
@@ -506,6 +506,109 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
       else
         rs = row_ok ? __ldg(p.sa + m) : 0.f;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(sp * 32) << 16) + (buf ? C::ACC1 : 0u);
+      // one 32 x 32 bf16 box: swizzled shared staging, then a TMA store
+      auto store_chunk = [&](const uint32_t (&pk)[16], int ocol) {
+        uint8_t* sbuf = staging + (nstore % C::NBUF) * STAGING_BYTES;
+        if (lane == 0) bulk_wait_group_read<C::NBUF - 1>();
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int sw = (j ^ ((lane >> 1) & 3)) << 4;
+          *reinterpret_cast<uint4*>(sbuf + lane * 64 + sw) =
+              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && slab_ok) {
+          tma_store_2d(&p.tmC, smem_u32(sbuf), ocol, row0);
+          bulk_commit_group();
+        }
+        ++nstore;
+      };
+      if constexpr (EPI == EPI_QKV) {
+        // One 128-column head per warp (head `half` of the tile).  Pass 1:
+        // the head's sum of squares (q and k heads); pass 2: re-read TMEM,
+        // normalize, weight, rotate the pairs, store.  Both passes recompute
+        // v = acc * scale + bias from TMEM instead of keeping 128 values.
+        const int h0 = nb * BN + QKV_HEAD_DIM * half;
+        const uint32_t hb = tbase + QKV_HEAD_DIM * half;
+        const bool hlive = h0 < p.N;
+        const bool normed = h0 < p.qk_cols;
+        const float* wgt = p.qk_w + (h0 < p.k_col0 ? 0 : QKV_HEAD_DIM);
+        const int64_t mrow = row_ok ? m : p.M - 1;  // padded rows read row M-1's angles
+        auto values = [&](int k, const uint32_t (&a)[32], float (&v)[32]) {
+          uint4 bp[4];
+          load_bf16x32_packed(p.bias + h0 + 32 * k, bp);
+          if constexpr (C::NV) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = fmaf(__uint_as_float(a[i]), rs, bf16x32_at(bp, i));
+          } else {
+            float sw[32];
+            load_f32x32(p.sw + h0 + 32 * k, sw);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              v[i] = fmaf(__uint_as_float(a[i]), rs * sw[i], bf16x32_at(bp, i));
+          }
+        };
+        float ss = 0.f;
+        if (hlive && normed) {
+#pragma unroll 1
+          for (int k = 0; k < 4; ++k) {
+            uint32_t a[32];
+            float v[32];
+            tmem_ld_32x32b_x32(hb + 32 * k, a);
+            tmem_wait_ld();
+            values(k, a, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
+          }
+        }
+        const float rn = normed ? rsqrtf(fmaf(ss, 1.f / QKV_HEAD_DIM, p.qk_eps)) : 1.f;
+#pragma unroll 1
+        for (int k = 0; k < 4; ++k) {
+          uint32_t a[32];
+          tmem_ld_32x32b_x32(hb + 32 * k, a);
+          tmem_wait_ld();
+          if (k == 3) {
+            // the whole head has been read: release this warp's share of both
+            // buffers (the overlap columns of NVFP4's 256-wide tiles included)
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              if (C::OVL) mbar_arrive_cluster(ovl_l0);
+              mbar_arrive_cluster(mapa_shared(smem_u32(&sb->acc_empty[buf]), 0));
+            }
+          }
+          if (!hlive) continue;
+          float v[32];
+          values(k, a, v);
+          if (normed) {
+            float w[32];
+            load_f32x32(wgt + 32 * k, w);
+            const float4* cp =
+                reinterpret_cast<const float4*>(p.rope_cos + mrow * (QKV_HEAD_DIM / 2) + 16 * k);
+            const float4* snp =
+                reinterpret_cast<const float4*>(p.rope_sin + mrow * (QKV_HEAD_DIM / 2) + 16 * k);
+#pragma unroll
+            for (int j4 = 0; j4 < 4; ++j4) {
+              const float4 c4 = __ldg(cp + j4), s4 = __ldg(snp + j4);
+              const float cs[4] = {c4.x, c4.y, c4.z, c4.w}, sn[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                const int i = 2 * (4 * j4 + t);
+                const float x0 = v[i] * rn * w[i], x1 = v[i + 1] * rn * w[i + 1];
+                v[i] = fmaf(x0, cs[t], -x1 * sn[t]);
+                v[i + 1] = fmaf(x0, sn[t], x1 * cs[t]);
+              }
+            }
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) pk[i >> 1] = pack_bf16x2(v[i], v[i + 1]);
+          store_chunk(pk, h0 + 32 * k);
+        }
+        continue;
+      }
       // chunk processed at step ci.  SwiGLU with overlapping buffers: the
       // shared columns are the up half of output chunks 2, 3 in buffer 0 and
       // the gate half of chunks 0, 1 in buffer 1; every warp holds exactly one
@@ -641,23 +744,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
           }
           continue;
         }
-        // ---- stage through swizzled shared memory, then one TMA store per warp
-        uint8_t* sbuf = staging + (nstore % C::NBUF) * STAGING_BYTES;
-        if (lane == 0) bulk_wait_group_read<C::NBUF - 1>();
-        __syncwarp();
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int sw = (j ^ ((lane >> 1) & 3)) << 4;
-          *reinterpret_cast<uint4*>(sbuf + lane * 64 + sw) =
-              make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && slab_ok) {
-          tma_store_2d(&p.tmC, smem_u32(sbuf), ocol, row0);
-          bulk_commit_group();
-        }
-        ++nstore;
+        store_chunk(packed, ocol);
       }
     }
     if (lane == 0) bulk_wait_group<0>();
@@ -720,7 +807,9 @@ cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t st) {
 
 int gemm_tile_n(int fmt, int epi) {
   if (fmt == 0) return Cfg<0, 2, EPI_BIAS>::BN;
-  return epi == EPI_SWIGLU ? Cfg<1, 2, EPI_SWIGLU>::BN : Cfg<1, 2, EPI_BIAS>::BN;
+  if (epi == EPI_SWIGLU) return Cfg<1, 2, EPI_SWIGLU>::BN;
+  if (epi == EPI_QKV) return Cfg<1, 2, EPI_QKV>::BN;
+  return Cfg<1, 2, EPI_BIAS>::BN;
 }
 
 cudaError_t launch_gemm(int fmt, int epi, int cg, int outq, const GemmParams& p, int num_sms,
@@ -740,11 +829,13 @@ cudaError_t launch_gemm(int fmt, int epi, int cg, int outq, const GemmParams& p,
   QLB_CASE(0, EPI_SWIGLU)
   QLB_CASE(0, EPI_GATED_RES)
   QLB_CASE(0, EPI_SPLIT)
+  QLB_CASE(0, EPI_QKV)
   QLB_CASE(1, EPI_BIAS)
   QLB_CASE(1, EPI_BIAS_GELU)
   QLB_CASE(1, EPI_SWIGLU)
   QLB_CASE(1, EPI_GATED_RES)
   QLB_CASE(1, EPI_SPLIT)
+  QLB_CASE(1, EPI_QKV)
   QLB_CASE_Q(EPI_BIAS)
   QLB_CASE_Q(EPI_BIAS_GELU)
   QLB_CASE_Q(EPI_SWIGLU)

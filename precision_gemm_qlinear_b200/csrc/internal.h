@@ -90,6 +90,9 @@ cudaError_t launch_quant_fp8_rows(const void* x, int64_t M, int64_t K, int64_t l
 cudaError_t launch_import_weights(int fmt, const void* codes, const void* scales, int64_t N,
                                   int64_t K, int64_t bn, uint8_t* wcodes, void* wscales, RowMap map,
                                   cudaStream_t st);
+// QKV epilogue norm weights (bf16 [128] each, null = all 1) -> fp32 [2][128].
+cudaError_t launch_qk_weights(const void* q_bf16, const void* k_bf16, float* dst,
+                              cudaStream_t st);
 cudaError_t launch_tensor_amax(const void* x, int64_t n_elems, uint32_t* amax_bits, int num_sms,
                                cudaStream_t st);
 // sf_layout: 0 = activation (A operand) atoms [sf_offset], 1 = weight (B
@@ -103,7 +106,11 @@ cudaError_t launch_permute_bias(const void* src, void* dst, int64_t N, RowMap ma
 // ------------------------------------------------------------------ GEMM
 
 enum Epi : int32_t { EPI_BIAS = 0, EPI_BIAS_GELU = 1, EPI_SWIGLU = 2, EPI_GATED_RES = 3,
-                     EPI_SPLIT = 4 };
+                     EPI_SPLIT = 4, EPI_QKV = 5 };
+
+// Head dimension of the QKV epilogue (per-head RMS normalization + rotary
+// embedding of q and k).
+constexpr int QKV_HEAD_DIM = 128;
 
 struct alignas(64) GemmParams {
   CUtensorMap tmA;  // activation codes [M, K(/2)] bytes, box 128 x 128 B, 128B swizzle
@@ -128,6 +135,14 @@ struct alignas(64) GemmParams {
   int32_t sf_kchunks_a, sfb_nstages;
   int32_t fault_mode;     // test hook: 0 = none
   int32_t gate_rows;      // gated residual: 0 = one gate [Nout]; else gate [M/gate_rows, Nout]
+  // QKV epilogue: columns [0, k_col0) are q heads, [k_col0, qk_cols) k heads,
+  // the rest v; qk_w = fp32 norm weights [2][128] (q then k); rope tables
+  // fp32 [M][64] (cos, sin of each token's angle per pair)
+  const float* qk_w;
+  const float* rope_cos;
+  const float* rope_sin;
+  int32_t k_col0, qk_cols;
+  float qk_eps;
   // NVFP4 output (instead of bf16): the epilogue's bf16 values quantized for a
   // next layer with K = Nout, against the tensor amax *q_amax supplied by the
   // caller.  Codes [M, Nout/2]; block scales in the sf_offset layout (padded

@@ -36,6 +36,8 @@ struct qlinear_s {
   float* wG;         // NVFP4 global scale (device scalar)
   uint32_t* wamax;   // NVFP4 amax word used while quantizing W
   __nv_bfloat16* bias;
+  float* qk_w;         // QKV epilogue: fp32 norm weights [2][128] (q, then k)
+  float qk_eps;        // QKV epilogue: RMS normalization epsilon
   RowMap map;
   int32_t fault_mode;  // test hook, see qlinear_debug_set_fault
   int32_t bn;          // N of the GEMM tile (256, or 224 for NVFP4 without SwiGLU)
@@ -53,7 +55,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 struct WsLayout {
-  size_t err, codes, scales, bias, total;
+  size_t err, codes, scales, bias, qk, total;
 };
 
 // Weight workspace: [control 256 B][codes][scales (+16 B tail for NVFP4)][bias]
@@ -72,6 +74,8 @@ WsLayout ws_layout(const ql_desc& d) {
   off = align_up(off + sc_bytes, 1024);
   L.bias = off;
   off = align_up(off + static_cast<size_t>(d.N) * 2, 1024);
+  L.qk = off;  // QKV epilogue: q and k norm weights (fp32, 2 x 128)
+  if (d.epi == QL_EPI_QKV_NORM_ROPE) off += 1024;
   L.total = off;
   return L;
 }
@@ -79,13 +83,15 @@ WsLayout ws_layout(const ql_desc& d) {
 ql_status check_desc(const ql_desc* d) {
   if (!d) return QL_ERR_INVALID_ARG;
   if (d->fmt != QL_FP8_E4M3 && d->fmt != QL_NVFP4) return QL_ERR_INVALID_ARG;
-  if (d->epi < QL_EPI_BIAS || d->epi > QL_EPI_SPLIT_BIAS_GELU) return QL_ERR_INVALID_ARG;
+  if (d->epi < QL_EPI_BIAS || d->epi > QL_EPI_QKV_NORM_ROPE) return QL_ERR_INVALID_ARG;
   if (d->flags != 0 || d->variant < 0 || d->variant > 2) return QL_ERR_INVALID_ARG;
   if (d->N < 1 || d->K < 1 || d->N > (1 << 24) || d->K > (1 << 24)) return QL_ERR_INVALID_ARG;
   if (d->N % 32 != 0) return QL_ERR_INVALID_ARG;
   if (d->fmt == QL_FP8_E4M3 && d->K % 16 != 0) return QL_ERR_INVALID_ARG;
   if (d->fmt == QL_NVFP4 && d->K % 32 != 0) return QL_ERR_INVALID_ARG;
   if (d->epi == QL_EPI_SWIGLU && d->N % 256 != 0) return QL_ERR_INVALID_ARG;
+  // q | k | v of 128-column heads, each part a whole number of 256-column tiles
+  if (d->epi == QL_EPI_QKV_NORM_ROPE && d->N % 768 != 0) return QL_ERR_INVALID_ARG;
   if (d->epi == QL_EPI_SPLIT_BIAS_GELU &&
       (d->split_col < 0 || d->split_col > d->N || d->split_col % 32 != 0))
     return QL_ERR_INVALID_ARG;
@@ -192,7 +198,8 @@ struct QOut {
 
 ql_status forward_impl(qlinear_t h, const void* codes, const void* scales, int64_t M,
                        const void* residual, const void* gate, int64_t gate_rows, void* out_bf16,
-                       const QOut* q, void* stream) {
+                       const QOut* q, const float* rope_cos, const float* rope_sin,
+                       void* stream) {
   if (!h || M < 0 || M > 0x7FFFFFFF) return QL_ERR_INVALID_ARG;
   if (M == 0) return QL_OK;
   if (!codes || !scales || (!q && !out_bf16)) return QL_ERR_INVALID_ARG;
@@ -200,6 +207,10 @@ ql_status forward_impl(qlinear_t h, const void* codes, const void* scales, int64
   if (gated && (!residual || !gate)) return QL_ERR_INVALID_ARG;
   if (gate_rows < 0 || gate_rows > 0x7FFFFFFF || (gate_rows > 0 && !gated))
     return QL_ERR_INVALID_ARG;
+  const bool qkv = h->d.epi == QL_EPI_QKV_NORM_ROPE;
+  if (qkv != (rope_cos != nullptr) || qkv != (rope_sin != nullptr)) return QL_ERR_INVALID_ARG;
+  if (qkv && (!aligned16(rope_cos) || !aligned16(rope_sin))) return QL_ERR_ALIGNMENT;
+  if (qkv && q) return QL_ERR_UNSUPPORTED;
   if (!aligned16(codes) || !aligned16(scales) || (!q && !aligned16(out_bf16)))
     return QL_ERR_ALIGNMENT;
   if (gated && (!aligned16(residual) || !aligned16(gate))) return QL_ERR_ALIGNMENT;
@@ -255,6 +266,12 @@ ql_status forward_impl(qlinear_t h, const void* codes, const void* scales, int64
   p.sfb_nstages = static_cast<int32_t>(sfb_stages(h->K));
   p.fault_mode = h->fault_mode;
   p.gate_rows = static_cast<int32_t>(gate_rows);
+  p.qk_w = h->qk_w;
+  p.rope_cos = rope_cos;
+  p.rope_sin = rope_sin;
+  p.k_col0 = static_cast<int32_t>(h->N / 3);
+  p.qk_cols = static_cast<int32_t>(2 * (h->N / 3));
+  p.qk_eps = h->qk_eps;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (q) {
     uint8_t* sf = static_cast<uint8_t*>(q->scales);
@@ -310,6 +327,8 @@ ql_status begin_create(const ql_desc* desc, const void* bias_bf16, void* weight_
   h->err = reinterpret_cast<uint32_t*>(h->ws + L.err);
   h->wcodes = h->ws + L.codes;
   h->bias = reinterpret_cast<__nv_bfloat16*>(h->ws + L.bias);
+  h->qk_w = reinterpret_cast<float*>(h->ws + L.qk);
+  h->qk_eps = 1e-6f;
   h->map.nout = h->Nout;
   h->map.mode = desc->epi == QL_EPI_SWIGLU ? 1 : 0;
   h->bn = gemm_tile_n(desc->fmt, desc->epi);
@@ -329,6 +348,8 @@ ql_status begin_create(const ql_desc* desc, const void* bias_bf16, void* weight_
 ql_status finish_create(qlinear_s* h, cudaError_t e, const void* bias_bf16, cudaStream_t st,
                         qlinear_t* out) {
   if (e == cudaSuccess) e = launch_permute_bias(bias_bf16, h->bias, h->N, h->map, st);
+  if (e == cudaSuccess && h->d.epi == QL_EPI_QKV_NORM_ROPE)
+    e = launch_qk_weights(nullptr, nullptr, h->qk_w, st);  // weights 1 until set
   if (e != cudaSuccess) {
     cudaGetLastError();
     delete h;
@@ -479,7 +500,32 @@ ql_status qlinear_quantize_act_noalloc(qlinear_t h, const void* x_bf16, int64_t 
 
 ql_status qlinear_forward(qlinear_t h, const void* codes, const void* scales, int64_t M,
                           const void* residual, const void* gate, void* out_bf16, void* stream) {
-  return forward_impl(h, codes, scales, M, residual, gate, 0, out_bf16, nullptr, stream);
+  return forward_impl(h, codes, scales, M, residual, gate, 0, out_bf16, nullptr, nullptr, nullptr,
+                      stream);
+}
+
+ql_status qlinear_forward_rope(qlinear_t h, const void* codes, const void* scales, int64_t M,
+                               const float* rope_cos, const float* rope_sin, void* out_bf16,
+                               void* stream) {
+  if (!rope_cos || !rope_sin) return QL_ERR_INVALID_ARG;
+  return forward_impl(h, codes, scales, M, nullptr, nullptr, 0, out_bf16, nullptr, rope_cos,
+                      rope_sin, stream);
+}
+
+ql_status qlinear_set_qk_norm(qlinear_t h, const void* q_weight_bf16, const void* k_weight_bf16,
+                              float eps, void* stream) {
+  if (!h || h->d.epi != QL_EPI_QKV_NORM_ROPE || !q_weight_bf16 || !k_weight_bf16)
+    return QL_ERR_INVALID_ARG;
+  if (!(eps >= 0.f && eps <= 3.4e38f)) return QL_ERR_INVALID_ARG;
+  if (!aligned16(q_weight_bf16) || !aligned16(k_weight_bf16)) return QL_ERR_ALIGNMENT;
+  cudaError_t e = launch_qk_weights(q_weight_bf16, k_weight_bf16, h->qk_w,
+                                    static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  h->qk_eps = eps;
+  return QL_OK;
 }
 
 ql_status qlinear_forward_gate_rows(qlinear_t h, const void* codes, const void* scales, int64_t M,
@@ -487,14 +533,15 @@ ql_status qlinear_forward_gate_rows(qlinear_t h, const void* codes, const void* 
                                     void* out_bf16, void* stream) {
   if (rows_per_gate < 1) return QL_ERR_INVALID_ARG;
   return forward_impl(h, codes, scales, M, residual, gate, rows_per_gate, out_bf16, nullptr,
-                      stream);
+                      nullptr, nullptr, stream);
 }
 
 ql_status qlinear_forward_nvfp4_out(qlinear_t h, const void* codes, const void* scales, int64_t M,
                                     const void* residual, const void* gate, const float* amax,
                                     void* out_codes, void* out_scales, void* stream) {
   const QOut q{out_codes, out_scales, amax};
-  return forward_impl(h, codes, scales, M, residual, gate, 0, nullptr, &q, stream);
+  return forward_impl(h, codes, scales, M, residual, gate, 0, nullptr, &q, nullptr, nullptr,
+                      stream);
 }
 
 ql_status qlinear_export_weights(qlinear_t h, void* codes_host, void* scales_host,

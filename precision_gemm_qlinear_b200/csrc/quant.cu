@@ -232,6 +232,16 @@ __global__ void import_block_scales_kernel(const uint8_t* __restrict__ src, uint
     *reinterpret_cast<uint32_t*>(sf + sfb_word_offset(row, g >> 2, g & 3, q4, nks, bn)) = word;
 }
 
+// QKV epilogue norm weights: bf16 q and k vectors of 128 -> fp32 [2][128]
+// (1.0 where a pointer is null).
+__global__ void qk_weights_kernel(const __nv_bfloat16* __restrict__ qw,
+                                  const __nv_bfloat16* __restrict__ kw, float* __restrict__ dst) {
+  const int i = threadIdx.x;  // 0..255
+  const __nv_bfloat16* src = i < QKV_HEAD_DIM ? qw : kw;
+  const int j = i & (QKV_HEAD_DIM - 1);
+  dst[i] = src ? __bfloat162float(src[j]) : 1.0f;
+}
+
 __global__ void permute_bias_kernel(const __nv_bfloat16* __restrict__ src,
                                     __nv_bfloat16* __restrict__ dst, int64_t N, RowMap map) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -310,6 +320,13 @@ cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx,
   cudaLaunchConfig_t c = pdl_config(static_cast<unsigned>(blocks), 256, 0, st, at, 0);
   return cudaLaunchKernelEx(&c, quant_nvfp4_kernel<4>, static_cast<const __nv_bfloat16*>(x), M, K,
                             ldx, q, sf, sf_layout, bn, nks, mpad, amax_bits, g_out, map);
+}
+
+cudaError_t launch_qk_weights(const void* q_bf16, const void* k_bf16, float* dst,
+                              cudaStream_t st) {
+  qk_weights_kernel<<<1, 2 * QKV_HEAD_DIM, 0, st>>>(static_cast<const __nv_bfloat16*>(q_bf16),
+                                                     static_cast<const __nv_bfloat16*>(k_bf16), dst);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_permute_bias(const void* src, void* dst, int64_t N, RowMap map,

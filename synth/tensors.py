@@ -13,7 +13,8 @@ Recipe (stated once, used everywhere):
 """
 import numpy as np
 
-TENSOR_IDS = {"x": 1, "w": 2, "bias": 3, "gate": 4, "residual": 5, "x2": 6, "w2": 7, "bias2": 8}
+TENSOR_IDS = {"x": 1, "w": 2, "bias": 3, "gate": 4, "residual": 5, "x2": 6, "w2": 7, "bias2": 8,
+              "q_norm": 9, "k_norm": 10}
 
 
 def rng_for(seed: int, tensor: str) -> np.random.Generator:

@@ -11,6 +11,8 @@ for real activations and weights (no checkpoint is used).
 from dataclasses import dataclass, field
 from typing import Optional
 
+import numpy as np
+
 from .tensors import draw
 
 
@@ -59,6 +61,10 @@ WORKLOADS = {
     "flux_qkv_fp8": Workload("flux_qkv_fp8", (
         Layer("fp8", 4608, 3072, 9216, "bias", _N01_OUT8),
     ), "FLUX-dev QKV projection, FP8, 4608x3072x9216, bias"),
+    "flux_qkv_normrope_fp8": Workload("flux_qkv_normrope_fp8", (
+        Layer("fp8", 4608, 3072, 9216, "qkv_norm_rope", _N01_OUT8),
+    ), "FLUX-dev QKV projection, FP8, 4608x3072x9216, q/k RMS norm per 128-column head + "
+       "rotary embedding, v bias"),
     "flux_mlp_fp8": Workload("flux_mlp_fp8", (
         Layer("fp8", 4608, 3072, 12288, "bias_gelu", _N01_OUT8),
         Layer("fp8", 4608, 12288, 3072, "bias_gated_residual", _N01, chained=True),
@@ -104,4 +110,13 @@ def make_inputs(layer: Layer, seed: int = 0, layer_index: int = 0, M: int = None
     if layer.epi == "bias_gated_residual":
         out["gate"] = draw("normal", (layer.Nout,), ws, "gate", mean=1.0, std=0.1)
         out["residual"] = draw("normal", (M, layer.Nout), seed, "residual", std=1.0)
+    if layer.epi == "qkv_norm_rope":
+        # norm weights near 1; rotary angles of a 1-D position grid with the
+        # usual geometric frequency ladder (base 10000) over the 64 pairs
+        out["q_norm"] = draw("normal", (128,), ws, "q_norm", mean=1.0, std=0.1)
+        out["k_norm"] = draw("normal", (128,), ws, "k_norm", mean=1.0, std=0.1)
+        pos = np.arange(M, dtype=np.float64)[:, None]
+        freq = 10000.0 ** (-np.arange(64, dtype=np.float64) / 64.0)[None, :]
+        out["rope_cos"] = np.cos(pos * freq).astype(np.float32)
+        out["rope_sin"] = np.sin(pos * freq).astype(np.float32)
     return out

@@ -44,6 +44,9 @@ def test_status_strings_and_version():
     ("fp8", "swiglu", 16384, 3072, True),
     ("fp8", "swiglu", 16416, 3072, False),   # SwiGLU needs N % 256
     ("fp8", "bias", 0, 3072, False),
+    ("fp8", "qkv_norm_rope", 9216, 3072, True),      # 3 x 24 heads of 128
+    ("nvfp4", "qkv_norm_rope", 9216, 3072, True),
+    ("fp8", "qkv_norm_rope", 9600, 3072, False),     # N % 768: q|k|v not tile-aligned
 ])
 def test_weight_bytes_shape_rules(fmt, epi, N, K, ok):
     s, n = ql.qlinear_weight_bytes(ql.make_desc(fmt, epi, N, K), check=False)
@@ -51,6 +54,13 @@ def test_weight_bytes_shape_rules(fmt, epi, N, K, ok):
     if ok:
         code = N * K if fmt == "fp8" else N * K // 2
         assert n >= code + 2 * N
+
+
+def test_unknown_epilogue_is_rejected():
+    d = ql.make_desc("fp8", "bias", 512, 256)
+    d.epi = 6
+    s, _ = ql.qlinear_weight_bytes(d, check=False)
+    assert s == _abi.QL_ERR_INVALID_ARG
 
 
 def test_split_col_rules():
