@@ -543,33 +543,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = fmaf(__uint_as_float(a[i]), rs, bf16x32_at(bp, i));
           } else {
-            float sw[32];
-            load_f32x32(p.sw + h0 + 32 * k, sw);
+            const float4* swp = reinterpret_cast<const float4*>(p.sw + h0 + 32 * k);
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              v[i] = fmaf(__uint_as_float(a[i]), rs * sw[i], bf16x32_at(bp, i));
+            for (int i4 = 0; i4 < 8; ++i4) {
+              const float4 s4 = __ldg(swp + i4);
+              const float sw4[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int i = 4 * i4 + j;
+                v[i] = fmaf(__uint_as_float(a[i]), rs * sw4[j], bf16x32_at(bp, i));
+              }
+            }
           }
         };
-        float ss = 0.f;
-        if (hlive && normed) {
-#pragma unroll 1
-          for (int k = 0; k < 4; ++k) {
-            uint32_t a[32];
-            float v[32];
-            tmem_ld_32x32b_x32(hb + 32 * k, a);
-            tmem_wait_ld();
-            values(k, a, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
+        if (!hlive) {
+          // a head past N (ragged N tile): nothing to read, release at once
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (C::OVL) mbar_arrive_cluster(ovl_l0);
+            mbar_arrive_cluster(mapa_shared(smem_u32(&sb->acc_empty[buf]), 0));
           }
+          continue;
         }
-        const float rn = normed ? rsqrtf(fmaf(ss, 1.f / QKV_HEAD_DIM, p.qk_eps)) : 1.f;
-#pragma unroll 1
-        for (int k = 0; k < 4; ++k) {
-          uint32_t a[32];
-          tmem_ld_32x32b_x32(hb + 32 * k, a);
+        // steps: 4 sum-of-squares chunks (q, k heads), then the 4 output
+        // chunks; the next step's TMEM load is in flight during each step
+        const int nsteps = normed ? 8 : 4;
+        uint32_t ha[32], hb2[32];
+        tmem_ld_32x32b_x32(hb, ha);
+        float ss = 0.f, rn = 1.f;
+        auto step = [&](int t, const uint32_t (&cur)[32], uint32_t (&nxt)[32]) {
+          const int k = t & 3;
           tmem_wait_ld();
-          if (k == 3) {
+          if (t + 1 < nsteps) tmem_ld_32x32b_x32(hb + 32 * ((t + 1) & 3), nxt);
+          if (t == nsteps - 1) {
             // the whole head has been read: release this warp's share of both
             // buffers (the overlap columns of NVFP4's 256-wide tiles included)
             tc_fence_before();
@@ -579,12 +586,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
               mbar_arrive_cluster(mapa_shared(smem_u32(&sb->acc_empty[buf]), 0));
             }
           }
-          if (!hlive) continue;
           float v[32];
-          values(k, a, v);
+          values(k, cur, v);
+          if (normed && t < 4) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
+            if (k == 3) rn = rsqrtf(fmaf(ss, 1.f / QKV_HEAD_DIM, p.qk_eps));
+            return;
+          }
           if (normed) {
-            float w[32];
-            load_f32x32(wgt + 32 * k, w);
+            const float4* wp = reinterpret_cast<const float4*>(wgt + 32 * k);
             const float4* cp =
                 reinterpret_cast<const float4*>(p.rope_cos + mrow * (QKV_HEAD_DIM / 2) + 16 * k);
             const float4* snp =
@@ -592,13 +603,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
 #pragma unroll
             for (int j4 = 0; j4 < 4; ++j4) {
               const float4 c4 = __ldg(cp + j4), s4 = __ldg(snp + j4);
+              const float4 w0 = __ldg(wp + 2 * j4), w1 = __ldg(wp + 2 * j4 + 1);
               const float cs[4] = {c4.x, c4.y, c4.z, c4.w}, sn[4] = {s4.x, s4.y, s4.z, s4.w};
+              const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                const int i = 2 * (4 * j4 + t);
-                const float x0 = v[i] * rn * w[i], x1 = v[i + 1] * rn * w[i + 1];
-                v[i] = fmaf(x0, cs[t], -x1 * sn[t]);
-                v[i + 1] = fmaf(x0, sn[t], x1 * cs[t]);
+              for (int tt = 0; tt < 4; ++tt) {
+                const int i = 2 * (4 * j4 + tt);
+                const float x0 = v[i] * rn * wv[2 * tt], x1 = v[i + 1] * rn * wv[2 * tt + 1];
+                v[i] = fmaf(x0, cs[tt], -x1 * sn[tt]);
+                v[i + 1] = fmaf(x0, sn[tt], x1 * cs[tt]);
               }
             }
           }
@@ -606,6 +619,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
 #pragma unroll
           for (int i = 0; i < 32; i += 2) pk[i >> 1] = pack_bf16x2(v[i], v[i + 1]);
           store_chunk(pk, h0 + 32 * k);
+        };
+#pragma unroll 1
+        for (int t = 0; t < nsteps; t += 2) {
+          step(t, ha, hb2);
+          step(t + 1, hb2, ha);
         }
         continue;
       }
