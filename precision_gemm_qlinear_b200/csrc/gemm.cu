@@ -651,13 +651,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
         // per-column and per-row operands: issued before the TMEM wait so the
         // two latencies overlap
         uint4 bias_a[4], bias_b[4], gate_a[4], res_a[4];
-        float sw_a[32], sw_b[32];
+        float sw_a[32];
         if (live) {
           load_bf16x32_packed(p.bias + ncol, bias_a);
           if constexpr (!C::NV) load_f32x32(p.sw + ncol, sw_a);
           if constexpr (EPI == EPI_SWIGLU) {
             load_bf16x32_packed(p.bias + ncol + 128, bias_b);
-            if constexpr (!C::NV) load_f32x32(p.sw + ncol + 128, sw_b);
           }
           if constexpr (EPI == EPI_GATED_RES) {
             // per-batch gates (CFG-batched tokens): row m uses gate row m / gate_rows
@@ -694,18 +693,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
           float v[32];
           if constexpr (EPI == EPI_SWIGLU) {
             float u[32];
+            // FP8: the up half's column scales are read in float4 pieces here
+            // (two preloaded 32-float arrays would not fit in registers)
+            const float4* swb = reinterpret_cast<const float4*>(p.sw + ncol + 128);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              float sa_, sb_;
-              if constexpr (C::NV) {
-                sa_ = rs;
-                sb_ = rs;
-              } else {
-                sa_ = rs * sw_a[i];
-                sb_ = rs * sw_b[i];
+            for (int i4 = 0; i4 < 8; ++i4) {
+              float sb4[4] = {rs, rs, rs, rs};
+              if constexpr (!C::NV) {
+                const float4 w4 = __ldg(swb + i4);
+                sb4[0] = rs * w4.x;
+                sb4[1] = rs * w4.y;
+                sb4[2] = rs * w4.z;
+                sb4[3] = rs * w4.w;
               }
-              v[i] = fmaf(__uint_as_float(ra[i]), sa_, bf16x32_at(bias_a, i));
-              u[i] = fmaf(__uint_as_float(accu[i]), sb_, bf16x32_at(bias_b, i));
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int i = 4 * i4 + j;
+                const float sa_ = C::NV ? rs : rs * sw_a[i];
+                v[i] = fmaf(__uint_as_float(ra[i]), sa_, bf16x32_at(bias_a, i));
+                u[i] = fmaf(__uint_as_float(accu[i]), sb4[j], bf16x32_at(bias_b, i));
+              }
             }
             silu_mul_32(v, u);
           } else {
