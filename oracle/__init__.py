@@ -45,6 +45,7 @@ def lib():
         L.or_gemm_nvfp4.argtypes = [P, P, ctypes.c_float, P, P, ctypes.c_float, i64, i64, P,
                                     i64, P]
         L.or_epilogue.argtypes = [ctypes.c_int, P, i64, i64, P, P, P, P, i64, P]
+        L.or_gemm_w8a16.argtypes = [P, P, P, i64, i64, P, i64, P]
         L.or_qkv_norm_rope.argtypes = [P, i64, i64, i64, P, P, P, P, P, P, ctypes.c_double, P]
         L.or_gelu_tanh.restype = ctypes.c_double
         L.or_gelu_tanh.argtypes = [ctypes.c_double]
@@ -144,6 +145,21 @@ def gemm_fp8(qa, sa, qw, sw, rows=None):
     return y
 
 
+def gemm_w8a16(x_bf16, qw, sw, rows=None):
+    """y = (sum_k x dec(qw)) * sw over the listed rows, x left in bf16
+    (weight-only quantization; C: or_gemm_w8a16)."""
+    x = _c(x_bf16, np.uint16)
+    qw = _c(qw, np.uint8)
+    sw = _c(sw, np.float32)
+    K = x.shape[1]
+    N = qw.shape[0]
+    assert qw.shape[1] == K
+    rows = np.arange(x.shape[0], dtype=np.int64) if rows is None else _c(rows, np.int64)
+    y = np.empty((len(rows), N), np.float64)
+    lib().or_gemm_w8a16(_p(x), _p(qw), _p(sw), K, N, _p(rows), len(rows), _p(y))
+    return y
+
+
 def gemm_nvfp4(qa, sfa, Ga, qw, sfw, Gw, rows=None):
     """Block-scaled NVFP4 GEMM over the listed rows (C: or_gemm_nvfp4)."""
     qa = _c(qa, np.uint8)
@@ -214,6 +230,10 @@ def qlinear_reference(fmt: str, epi: str, x_bf16, w_bf16, bias=None, residual=No
         qw, sw = quant_fp8_rows(w_bf16)
         y = gemm_fp8(qa, sa, qw, sw, rows)
         res = dict(qa=qa, sa=sa, qw=qw, sw=sw)
+    elif fmt == "w8a16":
+        qw, sw = quant_fp8_rows(w_bf16)
+        y = gemm_w8a16(x_bf16, qw, sw, rows)
+        res = dict(qw=qw, sw=sw)
     elif fmt == "nvfp4":
         qa, sfa, Ga = quant_nvfp4(x_bf16)
         qw, sfw, Gw = quant_nvfp4(w_bf16)

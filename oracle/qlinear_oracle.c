@@ -254,6 +254,28 @@ void or_gemm_fp8(const uint8_t* qa, const float* sa, const uint8_t* qw, const fl
   }
 }
 
+/* Weight-only GEMM: bf16 activations (not quantized) against decoded FP8
+ * weights, for the listed activation rows:
+ *   y[i, n] = ( sum_k x[row_i, k] * dec(qw[n, k]) ) * sw[n]
+ * x bf16 [*, K] row-major, qw [N, K].  A bf16 value times an E4M3 value has
+ * at most 12 significant bits, so each product is exact in binary64; the sum
+ * is rounded to binary64 (ordered by k). */
+void or_gemm_w8a16(const uint16_t* x, const uint8_t* qw, const float* sw, int64_t K, int64_t N,
+                   const int64_t* rows, int64_t nrows, double* y) {
+  double lut[256];
+  for (int c = 0; c < 256; ++c) lut[c] = or_e4m3_decode((uint8_t)c);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t i = 0; i < nrows; ++i) {
+    const uint16_t* a = x + rows[i] * K;
+    for (int64_t n = 0; n < N; ++n) {
+      const uint8_t* w = qw + n * K;
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += (double)bf16_to_f32(a[k]) * lut[w[k]];
+      y[i * N + n] = acc * (double)sw[n];
+    }
+  }
+}
+
 /* NVFP4 GEMM over the decoded codes, for the listed activation rows:
  *   y[i, n] = G_a * G_w * sum_b dec(sfa[row,b]) * dec(sfw[n,b])
  *                           * sum_{k in block b} dec(qa[row,k]) * dec(qw[n,k])

@@ -69,6 +69,39 @@ def test_fp8_gemm_sum_is_exact(orc):
             assert y[i, n] == math.fsum(dec[qa[i]] * dec[qw[n]])
 
 
+def test_w8a16_gemm_one_hot(orc):
+    # a bf16 one-hot row (value 1.0 at k) picks dec(qw[n, k]) * sw[n] exactly
+    K, N = 64, 8
+    x = np.zeros((2, K), np.uint16)
+    x[0, 7] = 0x3F80   # 1.0
+    x[1, 40] = 0xC000  # -2.0
+    qw = (np.arange(N * K, dtype=np.int64).reshape(N, K) * 7 % 256).astype(np.uint8) & 0x77
+    sw = np.array([2.0 ** -i for i in range(N)], np.float32)
+    y = orc.gemm_w8a16(x, qw, sw)
+    dec = np.array([orc.e4m3_decode(c) for c in range(256)])
+    assert np.array_equal(y[0], dec[qw[:, 7]] * sw)
+    assert np.array_equal(y[1], -2.0 * dec[qw[:, 40]] * sw)
+
+
+@pytest.mark.parametrize("K", [48, 3072])
+def test_w8a16_gemm_equals_fp8_gemm_on_fp8_valued_activations(orc, K):
+    # bf16 activations that are E4M3 values times a power of two per row: the
+    # weight-only GEMM must give exactly what the FP8 GEMM gives on the codes
+    # (every product and both sums are exact in binary64)
+    g = np.random.default_rng(K)
+    M, N = 4, 5
+    qa = g.integers(0, 256, (M, K), dtype=np.uint8)
+    qa[(qa & 0x7F) == 0x7F] = 0x31
+    qw = g.integers(0, 256, (N, K), dtype=np.uint8)
+    qw[(qw & 0x7F) == 0x7F] = 0x42
+    sa = np.array([2.0 ** (-3 + i) for i in range(M)], np.float32)
+    sw = g.uniform(0.5, 2.0, N).astype(np.float32)
+    dec = np.array([orc.e4m3_decode(c) for c in range(256)])
+    x = bf16_bits_from_f64(dec[qa] * sa[:, None].astype(np.float64))
+    assert np.array_equal(bf16_bits_to_f32(x).astype(np.float64), dec[qa] * sa[:, None])
+    assert np.array_equal(orc.gemm_w8a16(x, qw, sw), orc.gemm_fp8(qa, sa, qw, sw))
+
+
 @pytest.mark.parametrize("M,N,K", [(2, 3, 32), (4, 2, 64)])
 def test_nvfp4_gemm_exact_triple_loop(orc, M, N, K):
     g = np.random.default_rng(K + N)
