@@ -37,7 +37,7 @@ DEFAULT_WORKLOAD = "flux_qkv_fp8"
 L2_BYTES = 126 * 2 ** 20
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # nominal dense tensor-core ratios to bf16 (FP8 4.5 / 2.25 PF, FP4 9 / 2.25 PF)
-NOMINAL_RATIO = {"fp8": 2.0, "nvfp4": 4.0}
+NOMINAL_RATIO = {"fp8": 2.0, "nvfp4": 4.0, "w8a16": 1.0}  # w8a16 runs bf16 MMAs
 GEMM_SOURCES = ["precision_gemm_qlinear_b200/csrc/gemm.cu",
                 "precision_gemm_qlinear_b200/csrc/ptx.cuh",
                 "precision_gemm_qlinear_b200/csrc/internal.h"]
@@ -261,21 +261,23 @@ class Model:
             lay = d["lay"]
             fused_in = self.fused[i] and not unfused
             fused_out = i + 1 < len(layers) and self.fused[i + 1] and not unfused
-            if not fused_in:
+            w16 = self.wl.layers[i].fmt == "w8a16"  # activations stay bf16: x is the operand
+            if not fused_in and not w16:
                 lay.quantize(x, d["codes"], d["scales"], stream)
+            codes = x if w16 else d["codes"]
             M = self.wl.layers[i].M
             if gemm_events is not None:
                 gemm_events[i][0].record(stream)
             if fused_out:
                 nd = layers[i + 1]
-                lay.forward_nvfp4_out(d["codes"], d["scales"], M, self.amax_of(amax_from, i + 1),
+                lay.forward_nvfp4_out(codes, d["scales"], M, self.amax_of(amax_from, i + 1),
                                       nd["codes"], nd["scales"], d.get("residual"), d.get("gate"),
                                       stream)
             elif "rope_cos" in d:
-                lay.forward_rope(d["codes"], d["scales"], M, d["rope_cos"], d["rope_sin"],
-                                 d["out"], stream)
+                lay.forward_rope(codes, d["scales"], M, d["rope_cos"], d["rope_sin"], d["out"],
+                                 stream)
             else:
-                lay.forward_codes(d["codes"], d["scales"], M, d["out"], d.get("residual"),
+                lay.forward_codes(codes, d["scales"], M, d["out"], d.get("residual"),
                                   d.get("gate"), stream)
             if gemm_events is not None:
                 gemm_events[i][1].record(stream)
@@ -292,7 +294,7 @@ class Model:
     def launches_per_step(self):
         n = 0
         for j, layer in enumerate(self.wl.layers):
-            if not self.fused[j]:
+            if not self.fused[j] and layer.fmt != "w8a16":
                 n += 1 if layer.fmt == "fp8" else 2   # the quantize kernels
             n += 1                                     # the GEMM
         return n
@@ -312,8 +314,8 @@ def quant_roofline(model, stream, peaks, peak_src, min_ms=50.0):
     import torch
     out = []
     for j, layer in enumerate(model.wl.layers):
-        if model.fused[j]:
-            continue  # quantized by the previous layer's epilogue, no kernel of its own
+        if model.fused[j] or layer.fmt == "w8a16":
+            continue  # quantized by the previous layer's epilogue / not quantized at all
         def run(i):
             layers = model.sets[i % len(model.sets)]
             x = layers[0]["x"] if j == 0 else layers[j - 1]["out"]
@@ -345,33 +347,54 @@ def quant_roofline(model, stream, peaks, peak_src, min_ms=50.0):
     return out
 
 
+class OracleLayer:
+    """The oracle's path for one layer: weights quantized once (untimed), then
+    quantize + GEMM + epilogue over a slice of activation rows."""
+
+    def __init__(self, layer, inp, x):
+        import oracle
+        self.o, self.layer, self.inp, self.x = oracle, layer, inp, x
+        if layer.fmt in ("fp8", "w8a16"):
+            self.qw, self.sw = oracle.quant_fp8_rows(inp["w"])
+        else:
+            self.qw, self.sfw, self.gw = oracle.quant_nvfp4(inp["w"])
+            self.amax = oracle.tensor_amax(x)  # the tensor amax is over the whole input
+
+    def gemm(self, r0, rows):
+        o, L, xs = self.o, self.layer, self.x[r0:r0 + rows]
+        if L.fmt == "fp8":
+            qa, sa = o.quant_fp8_rows(xs)
+            return o.gemm_fp8(qa, sa, self.qw, self.sw)
+        if L.fmt == "w8a16":
+            return o.gemm_w8a16(xs, self.qw, self.sw)
+        qa, sfa, ga = o.quant_nvfp4(xs, amax=self.amax)
+        return o.gemm_nvfp4(qa, sfa, ga, self.qw, self.sfw, self.gw)
+
+    def run(self, r0, rows):
+        o, L, inp = self.o, self.layer, self.inp
+        y = self.gemm(r0, rows)
+        if L.epi == "qkv_norm_rope":
+            return o.qkv_norm_rope(y, inp["bias"], inp["q_norm"], inp["k_norm"],
+                                   inp["rope_cos"][r0:r0 + rows], inp["rope_sin"][r0:r0 + rows])
+        res = inp.get("residual")
+        return o.epilogue(L.epi, y, bias=inp["bias"], split_col=L.split_col,
+                          residual=None if res is None else res[r0:r0 + rows],
+                          gate=inp.get("gate"))
+
+
 def cpu_baseline(wl, seconds):
     """Time the oracle (as it stands) on a bounded row sample of the workload's
     first layer; returns TFLOP/s-equivalent and a description."""
-    import oracle
     layer = wl.layers[0]
     inp = make_inputs(layer, seed=0)
     x = inp.get("x")
     if x is None:  # chained input: use a synthetic bf16 stand-in of the same shape
         x = make_inputs(wl.layers[0], seed=0)["x"]
-    # weights quantized once, untimed (not part of the per-step path)
-    if layer.fmt == "fp8":
-        qw, sw = oracle.quant_fp8_rows(inp["w"])
-    else:
-        qw, sfw, gw = oracle.quant_nvfp4(inp["w"])
-        amax = oracle.tensor_amax(x)
+    ol = OracleLayer(layer, inp, x)  # weights quantized once, untimed
 
     def run(rows):
         t0 = time.perf_counter()
-        xs = x[:rows]
-        if layer.fmt == "fp8":
-            qa, sa = oracle.quant_fp8_rows(xs)
-            y = oracle.gemm_fp8(qa, sa, qw, sw)
-        else:
-            qa, sfa, ga = oracle.quant_nvfp4(xs, amax=amax)
-            y = oracle.gemm_nvfp4(qa, sfa, ga, qw, sfw, gw)
-        oracle.epilogue(layer.epi, y, bias=inp["bias"], residual=inp.get("residual"),
-                        gate=inp.get("gate"), split_col=layer.split_col)
+        ol.run(0, rows)
         return time.perf_counter() - t0
 
     probe = 4
@@ -382,7 +405,7 @@ def cpu_baseline(wl, seconds):
     rows = int(max(1, min(layer.M, probe * seconds / max(t, 1e-6))))
     dt = run(rows) if rows != probe else t
     flops = 2.0 * rows * layer.N * layer.K
-    return flops / dt / 1e12, rows, dt, oracle.num_threads()
+    return flops / dt / 1e12, rows, dt, ol.o.num_threads()
 
 
 def main_ours(args):
@@ -401,7 +424,7 @@ def main_ours(args):
 
     per_set = 0
     for layer in wl.layers:
-        kb = layer.K if layer.fmt == "fp8" else layer.K // 2
+        kb = layer.K // 2 if layer.fmt == "nvfp4" else layer.K
         per_set += layer.M * layer.K * 2 + layer.N * kb + layer.M * (
             layer.N // 2 if layer.epi == "swiglu" else layer.N) * 2
     nsets = args.sets or max(2, int(np.ceil(2 * L2_BYTES / per_set)) + 1)
@@ -491,7 +514,8 @@ def main_ours(args):
             "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": wl.layers[0].fmt if len(set(l.fmt for l in wl.layers)) == 1 else "mixed",
+            "dtype": ({"fp8": "fp8", "nvfp4": "nvfp4", "w8a16": "bf16"}[wl.layers[0].fmt]
+                      if len(set(l.fmt for l in wl.layers)) == 1 else "mixed"),
             "data": "synthetic (seeded FLUX-shaped activations and random-init weights)",
             "config": {"workload": wl.name, "desc": wl.note,
                        "layers": [dict(fmt=l.fmt, M=l.M, K=l.K, N=l.N, epi=l.epi) for l in wl.layers],
@@ -582,48 +606,24 @@ def main_reference(args):
     layer = wl.layers[0]
     inp = make_inputs(layer, seed=0)
     x = inp.get("x")
-    if layer.fmt == "fp8":
-        qw, sw = oracle.quant_fp8_rows(inp["w"])
-    else:
-        qw, sfw, gw = oracle.quant_nvfp4(inp["w"])
-        amax = oracle.tensor_amax(x)
+    ol = OracleLayer(layer, inp, x)
     # bounded per-step row sample so that warm-up + steps finish in a few minutes
     per_row = 2.0 * layer.N * layer.K
     budget_s = 150.0 / max(1, args.steps + args.warmup)
-    rows = 1
     t0 = time.perf_counter()
-    if layer.fmt == "fp8":
-        qa, sa = oracle.quant_fp8_rows(x[:1])
-        oracle.gemm_fp8(qa, sa, qw, sw)
-    else:
-        qa, sfa, ga = oracle.quant_nvfp4(x[:1], amax=amax)
-        oracle.gemm_nvfp4(qa, sfa, ga, qw, sfw, gw)
+    ol.gemm(0, 1)
     t1 = time.perf_counter() - t0
     probe = 1
     while t1 < 0.5 and probe < layer.M:  # size the per-step sample from a timed probe
         probe = min(layer.M, probe * 4)
         t0 = time.perf_counter()
-        if layer.fmt == "fp8":
-            qa, sa = oracle.quant_fp8_rows(x[:probe])
-            oracle.gemm_fp8(qa, sa, qw, sw)
-        else:
-            qa, sfa, ga = oracle.quant_nvfp4(x[:probe], amax=amax)
-            oracle.gemm_nvfp4(qa, sfa, ga, qw, sfw, gw)
+        ol.gemm(0, probe)
         t1 = time.perf_counter() - t0
     rows = int(max(1, min(layer.M, probe * budget_s / max(t1, 1e-6))))
 
     def step(i):
         r0 = (i * rows) % max(1, layer.M - rows + 1)
-        xs = x[r0:r0 + rows]
-        if layer.fmt == "fp8":
-            qa, sa = oracle.quant_fp8_rows(xs)
-            y = oracle.gemm_fp8(qa, sa, qw, sw)
-        else:
-            qa, sfa, ga = oracle.quant_nvfp4(xs, amax=amax)
-            y = oracle.gemm_nvfp4(qa, sfa, ga, qw, sfw, gw)
-        oracle.epilogue(layer.epi, y, bias=inp["bias"], split_col=layer.split_col,
-                        residual=None if "residual" not in inp else inp["residual"][r0:r0 + rows],
-                        gate=inp.get("gate"))
+        ol.run(r0, rows)
 
     for i in range(args.warmup):
         step(i)

@@ -61,7 +61,13 @@ typedef enum {
   QL_ERR_TIMEOUT = 5      /* a device-side bounded wait expired                */
 } ql_status;
 
-typedef enum { QL_FP8_E4M3 = 0, QL_NVFP4 = 1 } ql_format;
+/* QL_W8A16: weight-only quantization -- FP8-E4M3 weights (per output channel
+ * scales, as QL_FP8_E4M3) against bf16 activations that are not quantized;
+ * the GEMM expands each FP8 weight stage to bf16 in shared memory and runs
+ * bf16 tensor-core MMAs.  Its "codes" are the bf16 activations themselves
+ * ([M, K], qlinear_quantize_act copies them; forward may be given x directly)
+ * and it has no activation scales (scales may be NULL in qlinear_forward). */
+typedef enum { QL_FP8_E4M3 = 0, QL_NVFP4 = 1, QL_W8A16 = 2 } ql_format;
 
 typedef enum {
   QL_EPI_BIAS = 0,                 /* out = y + b                                  */
@@ -89,7 +95,7 @@ typedef struct {
 } ql_desc;
 
 /* Shape rules (QL_ERR_INVALID_ARG otherwise):
- *   FP8  : K % 16 == 0, N % 32 == 0;  NVFP4: K % 32 == 0, N % 32 == 0;
+ *   FP8, W8A16: K % 16 == 0, N % 32 == 0;  NVFP4: K % 32 == 0, N % 32 == 0;
  *   SwiGLU: N % 256 == 0;  QKV with norm + RoPE: N % 768 == 0;  1 <= K <= 2^24, 1 <= N <= 2^24, 0 <= M <= 2^31-1;
  *   split_col % 32 == 0 for the split epilogue.
  */

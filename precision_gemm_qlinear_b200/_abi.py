@@ -11,8 +11,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libqlinear_b200.so")
 
 QL_OK, QL_ERR_INVALID_ARG, QL_ERR_ALIGNMENT, QL_ERR_UNSUPPORTED, QL_ERR_CUDA, QL_ERR_TIMEOUT = range(6)
-QL_FP8_E4M3, QL_NVFP4 = 0, 1
-FORMATS = {"fp8": QL_FP8_E4M3, "nvfp4": QL_NVFP4}
+QL_FP8_E4M3, QL_NVFP4, QL_W8A16 = 0, 1, 2
+FORMATS = {"fp8": QL_FP8_E4M3, "nvfp4": QL_NVFP4, "w8a16": QL_W8A16}
 EPILOGUES = {"bias": 0, "bias_gelu": 1, "swiglu": 2, "bias_gated_residual": 3,
              "split_bias_gelu": 4, "qkv_norm_rope": 5}
 

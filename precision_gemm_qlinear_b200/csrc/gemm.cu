@@ -63,6 +63,10 @@ constexpr uint32_t idesc_f8() {
   return (1u << 4) | (0u << 7) | (0u << 10) | ((BN >> 3) << 17) | (((BM * CG) >> 4) << 24);
 }
 template <int CG, int BN>
+constexpr uint32_t idesc_bf16() {  // kind::f16 with A and B bf16, fp32 accumulate
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | (((BM * CG) >> 4) << 24);
+}
+template <int CG, int BN>
 constexpr uint32_t idesc_f4() {
   return (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | (((BM * CG) >> 4) << 24);
 }
@@ -70,7 +74,11 @@ constexpr uint32_t idesc_f4() {
 template <int FMT, int CG, int EPI>
 struct Cfg {
   static constexpr bool NV = (FMT == 1);
+  // FMT 2: bf16 activations x FP8 weights.  The FP8 weight stage lands raw
+  // (B8) and converter warps expand it to bf16 in the MMA's B layout.
+  static constexpr bool W16 = (FMT == 2);
   static constexpr bool PAIR = (CG == 2);
+  static constexpr int THREADS = W16 ? 384 : 320;
   // Tile N: 256, except NVFP4 without SwiGLU, where 224 lets two fp32
   // accumulators (2 x 224 TMEM columns) and the 48 scale-factor columns fit
   // in the 512 columns side by side.
@@ -78,15 +86,16 @@ struct Cfg {
   static constexpr int B_BYTES = (BN / CG) * BK_BYTES;  // this CTA's rows of B
   static constexpr int SFA_BYTES = NV ? 2048 : 0;       // 4 atoms (one per MMA K step)
   static constexpr int SFB_BYTES = NV ? 16384 : 0;      // 4 replicated 4 KB chunks (all 256 B rows)
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = NV ? (PAIR ? 4 : 3) : (PAIR ? 6 : 4);
+  static constexpr int B8_BYTES = W16 ? (BN / CG) * 64 : 0;  // raw FP8 weights, 64 per row
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES + B8_BYTES;
+  static constexpr int STAGES = NV ? (PAIR ? 4 : 3) : (W16 ? (PAIR ? 4 : 3) : (PAIR ? 6 : 4));
   // staging buffers per epilogue warp: two unless that breaks the budget
   static constexpr int NBUF =
-      (STAGES * STAGE_BYTES + NUM_EPI_WARPS * 2 * STAGING_BYTES + 256 + 1024 <= 232448) ? 2 : 1;
+      (STAGES * STAGE_BYTES + NUM_EPI_WARPS * 2 * STAGING_BYTES + 512 + 1024 <= 232448) ? 2 : 1;
   static constexpr int STAGING_OFF = STAGES * STAGE_BYTES;
   static constexpr int BAR_OFF = STAGING_OFF + NUM_EPI_WARPS * NBUF * STAGING_BYTES;
-  static_assert(BAR_OFF + 256 + 1024 <= 232448, "shared memory budget");
-  static constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
+  static_assert(BAR_OFF + 512 + 1024 <= 232448, "shared memory budget");
+  static constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;  // + barriers + alignment slack
   // TMEM columns: FP8 -> two disjoint 256-column accumulators.  NVFP4 ->
   // the scale factors of the current stage live in [448, 496) (A in 4 x 4
   // columns, B in 4 x 8, one group per 64-element MMA step); with N = 224 the
@@ -107,11 +116,13 @@ struct SmemBars {
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t ovl_free;
+  uint64_t b8_full[8];    // FMT 2: raw weight stage landed (this CTA)
+  uint64_t conv_done[8];  // FMT 2: weight stage converted (both CTAs, at the leader)
   uint64_t drain;
   uint32_t tmem_base;
   volatile int32_t abort_flag;
 };
-static_assert(sizeof(SmemBars) <= 256, "barrier block exceeds its reservation");
+static_assert(sizeof(SmemBars) <= 512, "barrier block exceeds its reservation");
 
 __device__ __forceinline__ void tile_coords(int t, const GemmParams& p, int& mb, int& nb) {
   const int per_group = p.group_m * p.tiles_n;
@@ -239,7 +250,7 @@ __device__ __forceinline__ void load_f32x32(const float* p, float (&o)[32]) {
 // OQ = 1: the epilogue writes NVFP4 codes and block scales for the next
 // layer instead of bf16 (see GemmParams::q_*).
 template <int FMT, int EPI, int CG, int OQ>
-__global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(FMT == 2 ? 384 : 320, 1) qgemm_kernel(const __grid_constant__ GemmParams p) {
   using C = Cfg<FMT, CG, EPI>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
@@ -263,6 +274,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
       mbar_init(smem_u32(&sb->acc_empty[b]), C::EPI_ARRIVALS);
     }
     mbar_init(smem_u32(&sb->ovl_free), C::EPI_ARRIVALS);
+    for (int s = 0; s < 8; ++s) {
+      mbar_init(smem_u32(&sb->b8_full[s]), 1);
+      mbar_init(smem_u32(&sb->conv_done[s]), 2 * CG);
+    }
     mbar_init(smem_u32(&sb->drain), 1);
     sb->abort_flag = 0;
     fence_mbarrier_init();
@@ -318,9 +333,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
           } else {
             if constexpr (C::PAIR) {
               const uint32_t lfb = mapa_shared(fb, 0);  // the leader's full barrier
+              if constexpr (C::W16) {
+                // bf16 activations (64 elements = 128 bytes per stage) counted
+                // at the leader; the raw FP8 weights on this CTA's own barrier,
+                // where this CTA's converter warps wait for them
+                if (rank == 0) mbar_arrive_expect_tx(fb, 2 * A_BYTES);
+                tma_load_2d_pair(smem_u32(st), &p.tmA, lfb, kb * 64, a_row);
+                const uint32_t xb = smem_u32(&sb->b8_full[stage]);
+                mbar_arrive_expect_tx(xb, C::B8_BYTES);
+                tma_load_2d(smem_u32(st + A_BYTES + C::B_BYTES), &p.tmB, xb, kb * 64, b_row);
+              } else {
               if (rank == 0) mbar_arrive_expect_tx(fb, 2 * C::STAGE_BYTES);
               tma_load_2d_pair(smem_u32(st), &p.tmA, lfb, kb * BK_BYTES, a_row);
               tma_load_2d_pair(smem_u32(st + A_BYTES), &p.tmB, lfb, kb * BK_BYTES, b_row);
+              }
               if constexpr (C::NV) {
                 // scales through 2-D maps of 2048-byte rows (uint64 x 256): the
                 // A atoms of this CTA's 128 rows (one row of the map) and the
@@ -333,9 +359,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
                                  8 * (nb * p.sfb_nstages + kb));
               }
             } else {
+              if constexpr (C::W16) {
+                mbar_arrive_expect_tx(fb, A_BYTES);
+                tma_load_2d(smem_u32(st), &p.tmA, fb, kb * 64, a_row);
+                const uint32_t xb = smem_u32(&sb->b8_full[stage]);
+                mbar_arrive_expect_tx(xb, C::B8_BYTES);
+                tma_load_2d(smem_u32(st + A_BYTES + C::B_BYTES), &p.tmB, xb, kb * 64, b_row);
+              } else {
               mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
               tma_load_2d(smem_u32(st), &p.tmA, fb, kb * BK_BYTES, a_row);
               tma_load_2d(smem_u32(st + A_BYTES), &p.tmB, fb, kb * BK_BYTES, b_row);
+              }
               if constexpr (C::NV) {
                 const uint8_t* sfa =
                     p.sfa + (static_cast<int64_t>(mb) * p.sf_kchunks_a + kb * 4) * 512;
@@ -355,14 +389,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
           }
         }
       }
-      if (sb->abort_flag && rank == 0) {
-        // let every load counted on this CTA's full barriers land before exit
+      if (sb->abort_flag && (rank == 0 || C::W16)) {
+        // let every load counted on this CTA's barriers land before exit (the
+        // leader's full barriers count both CTAs' loads; FMT 2's raw weight
+        // loads are counted on each CTA's own b8_full barriers)
         for (int s = 0; s < C::STAGES; ++s)
           if (issued_mask & (1u << s)) {
-            const uint32_t a = smem_u32(&sb->full[s]);
             const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(a, (issued_phase >> s) & 1) &&
-                   globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
+            if (rank == 0) {
+              const uint32_t a = smem_u32(&sb->full[s]);
+              while (!mbar_try_wait(a, (issued_phase >> s) & 1) &&
+                     globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
+              }
+            }
+            if constexpr (C::W16) {
+              const uint32_t x = smem_u32(&sb->b8_full[s]);
+              while (!mbar_try_wait(x, (issued_phase >> s) & 1) &&
+                     globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
+              }
             }
           }
       }
@@ -400,6 +444,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
             ok = false;
             break;
           }
+          if constexpr (C::W16) {
+            // both CTAs' converter warps have written this stage's bf16 B
+            if (!wait_bar(&sb->conv_done[stage], phase, sb, p.err, ERR_WAIT_MMA)) {
+              ok = false;
+              break;
+            }
+          }
           tc_fence_after();
           // this stage's descriptors: the stage-0 descriptors advanced by the
           // stage offset in the 16-byte start-address field
@@ -433,6 +484,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
               else
                 mma_mxf4nvf4(d_tmem, ad, bd, idesc_f4<CG, BN>(), t_sfa + 4 * j, t_sfb + 8 * j,
                              acc);
+            } else if constexpr (C::W16) {
+              if constexpr (C::PAIR)
+                mma_bf16_pair(d_tmem, ad, bd, idesc_bf16<CG, BN>(), acc);
+              else
+                mma_bf16(d_tmem, ad, bd, idesc_bf16<CG, BN>(), acc);
             } else {
               if constexpr (C::PAIR)
                 mma_f8f6f4_pair(d_tmem, ad, bd, idesc_f8<CG, BN>(), acc);
@@ -465,6 +521,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
         const uint32_t a = smem_u32(&sb->drain);
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
+        }
+      }
+    }
+  } else if (warp >= 2 + NUM_EPI_WARPS) {
+    // ------------------------ FMT 2: FP8 weight stage -> bf16 MMA operand
+    // Two warps per CTA.  Row r of this CTA's BN/CG weight rows: 64 E4M3
+    // bytes at B8 + 64 r become 64 bf16 (exact) in the 128-byte-swizzled
+    // K-major layout the MMA descriptor reads: 16-byte chunk c of row r at
+    // B + 128 r + ((c ^ (r & 7)) << 4) (the B region is 1024-byte aligned).
+    if constexpr (C::W16) {
+      const int ct = threadIdx.x - 32 * (2 + NUM_EPI_WARPS);  // 0..63
+      const uint32_t done_l0 = mapa_shared(smem_u32(&sb->conv_done[0]), 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = unit; t < num_tiles && ok; t += nunits) {
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!wait_bar(&sb->b8_full[stage], phase, sb, p.err, ERR_WAIT_EPI)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + stage * C::STAGE_BYTES;
+          const uint8_t* b8 = st + A_BYTES + C::B_BYTES;
+          uint8_t* bb = st + A_BYTES;
+#pragma unroll
+          for (int rr = 0; rr < (BN / CG) / 64; ++rr) {
+            const int r = ct + 64 * rr;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint4 c = *reinterpret_cast<const uint4*>(b8 + 64 * r + 16 * j);
+              const uint4 lo = make_uint4(e4m3x2_to_bf16x2(c.x), e4m3x2_to_bf16x2(c.x >> 16),
+                                          e4m3x2_to_bf16x2(c.y), e4m3x2_to_bf16x2(c.y >> 16));
+              const uint4 hi = make_uint4(e4m3x2_to_bf16x2(c.z), e4m3x2_to_bf16x2(c.z >> 16),
+                                          e4m3x2_to_bf16x2(c.w), e4m3x2_to_bf16x2(c.w >> 16));
+              *reinterpret_cast<uint4*>(bb + 128 * r + (((2 * j) ^ (r & 7)) << 4)) = lo;
+              *reinterpret_cast<uint4*>(bb + 128 * r + (((2 * j + 1) ^ (r & 7)) << 4)) = hi;
+            }
+          }
+          fence_proxy_async_smem();  // generic-proxy writes -> the tensor core's reads
+          __syncwarp();
+          if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(done_l0 + 8u * stage);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
         }
       }
     }
@@ -503,6 +604,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) qgemm_kernel(const __grid_cons
       float rs;
       if constexpr (C::NV)
         rs = __ldg(p.ga) * __ldg(p.gw);
+      else if constexpr (C::W16)
+        rs = 1.f;  // bf16 activations carry no scale
       else
         rs = row_ok ? __ldg(p.sa + m) : 0.f;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(sp * 32) << 16) + (buf ? C::ACC1 : 0u);
@@ -813,7 +916,7 @@ cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t st) {
   if (grid <= 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
@@ -832,6 +935,7 @@ cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t st) {
 
 int gemm_tile_n(int fmt, int epi) {
   if (fmt == 0) return Cfg<0, 2, EPI_BIAS>::BN;
+  if (fmt == 2) return Cfg<2, 2, EPI_BIAS>::BN;
   if (epi == EPI_SWIGLU) return Cfg<1, 2, EPI_SWIGLU>::BN;
   if (epi == EPI_QKV) return Cfg<1, 2, EPI_QKV>::BN;
   return Cfg<1, 2, EPI_BIAS>::BN;
@@ -866,6 +970,12 @@ cudaError_t launch_gemm(int fmt, int epi, int cg, int outq, const GemmParams& p,
   QLB_CASE_Q(EPI_SWIGLU)
   QLB_CASE_Q(EPI_GATED_RES)
   QLB_CASE_Q(EPI_SPLIT)
+  QLB_CASE(2, EPI_BIAS)
+  QLB_CASE(2, EPI_BIAS_GELU)
+  QLB_CASE(2, EPI_SWIGLU)
+  QLB_CASE(2, EPI_GATED_RES)
+  QLB_CASE(2, EPI_SPLIT)
+  QLB_CASE(2, EPI_QKV)
 #undef QLB_CASE
 #undef QLB_CASE_Q
   return cudaErrorInvalidValue;

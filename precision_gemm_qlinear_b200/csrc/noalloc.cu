@@ -99,6 +99,15 @@ __global__ void __launch_bounds__(256) reduce_amax_kernel(const uint32_t* __rest
 
 ql_status quantize_act_noalloc(int fmt, int64_t K, int num_sms, const void* x, int64_t M,
                                void* codes, void* scales, cudaStream_t st) {
+  if (fmt == QL_W8A16) {
+    // weight-only layers keep bf16 activations: a copy, no working memory
+    if (cudaMemcpyAsync(codes, x, static_cast<size_t>(M) * K * 2, cudaMemcpyDeviceToDevice, st) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return QL_ERR_CUDA;
+    }
+    return QL_OK;
+  }
   if (fmt == QL_FP8_E4M3) {
     // per-token FP8 is a single pass with no working memory at all
     cudaError_t e = launch_quant_fp8_rows(x, M, K, K, static_cast<uint8_t*>(codes),

@@ -82,12 +82,13 @@ WsLayout ws_layout(const ql_desc& d) {
 
 ql_status check_desc(const ql_desc* d) {
   if (!d) return QL_ERR_INVALID_ARG;
-  if (d->fmt != QL_FP8_E4M3 && d->fmt != QL_NVFP4) return QL_ERR_INVALID_ARG;
+  if (d->fmt != QL_FP8_E4M3 && d->fmt != QL_NVFP4 && d->fmt != QL_W8A16)
+    return QL_ERR_INVALID_ARG;
   if (d->epi < QL_EPI_BIAS || d->epi > QL_EPI_QKV_NORM_ROPE) return QL_ERR_INVALID_ARG;
   if (d->flags != 0 || d->variant < 0 || d->variant > 2) return QL_ERR_INVALID_ARG;
   if (d->N < 1 || d->K < 1 || d->N > (1 << 24) || d->K > (1 << 24)) return QL_ERR_INVALID_ARG;
   if (d->N % 32 != 0) return QL_ERR_INVALID_ARG;
-  if (d->fmt == QL_FP8_E4M3 && d->K % 16 != 0) return QL_ERR_INVALID_ARG;
+  if (d->fmt != QL_NVFP4 && d->K % 16 != 0) return QL_ERR_INVALID_ARG;
   if (d->fmt == QL_NVFP4 && d->K % 32 != 0) return QL_ERR_INVALID_ARG;
   if (d->epi == QL_EPI_SWIGLU && d->N % 256 != 0) return QL_ERR_INVALID_ARG;
   // q | k | v of 128-column heads, each part a whole number of 256-column tiles
@@ -177,11 +178,13 @@ ql_status from_cuda(cudaError_t e) {
 }
 
 size_t act_code_bytes(const qlinear_s* h, int64_t M) {
+  if (h->d.fmt == QL_W8A16) return static_cast<size_t>(M) * h->K * 2;  // the bf16 values
   return h->d.fmt == QL_NVFP4 ? static_cast<size_t>(M) * h->K / 2 : static_cast<size_t>(M) * h->K;
 }
 
 size_t act_scale_bytes(const qlinear_s* h, int64_t M) {
   if (h->d.fmt == QL_NVFP4) return static_cast<size_t>(sf_bytes(M, h->K)) + 16;
+  if (h->d.fmt == QL_W8A16) return 16;  // no activation scales
   return align_up(static_cast<size_t>(M) * 4, 16);
 }
 
@@ -202,7 +205,8 @@ ql_status forward_impl(qlinear_t h, const void* codes, const void* scales, int64
                        void* stream) {
   if (!h || M < 0 || M > 0x7FFFFFFF) return QL_ERR_INVALID_ARG;
   if (M == 0) return QL_OK;
-  if (!codes || !scales || (!q && !out_bf16)) return QL_ERR_INVALID_ARG;
+  const bool w16 = h->d.fmt == QL_W8A16;  // activations are bf16, no scales
+  if (!codes || (!scales && !w16) || (!q && !out_bf16)) return QL_ERR_INVALID_ARG;
   const bool gated = h->d.epi == QL_EPI_BIAS_GATED_RESIDUAL;
   if (gated && (!residual || !gate)) return QL_ERR_INVALID_ARG;
   if (gate_rows < 0 || gate_rows > 0x7FFFFFFF || (gate_rows > 0 && !gated))
@@ -226,12 +230,14 @@ ql_status forward_impl(qlinear_t h, const void* codes, const void* scales, int64
 
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
-  const uint64_t kbytes = nv ? h->K / 2 : h->K;
+  const uint64_t kbytes = nv ? h->K / 2 : (w16 ? h->K * 2 : h->K);  // A bytes per row
   // one CTA per 128-row tile for a single M tile, else CTA pairs on 256 rows
   const int cg = h->d.variant == 1 ? 1 : (h->d.variant == 2 ? 2 : (M > 128 ? 2 : 1));
-  if (!make_tmap(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, kbytes, M, kbytes, 128, 128,
-                 CU_TENSOR_MAP_SWIZZLE_128B))
-    return QL_ERR_CUDA;
+  const bool amap = w16 ? make_tmap(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, codes, h->K, M, kbytes,
+                                    64, 128, CU_TENSOR_MAP_SWIZZLE_128B)
+                        : make_tmap(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, kbytes, M, kbytes,
+                                    128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!amap) return QL_ERR_CUDA;
   if (!q && !make_tmap(&p.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out_bf16, h->Nout, M,
                        h->Nout * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return QL_ERR_CUDA;
@@ -332,7 +338,7 @@ ql_status begin_create(const ql_desc* desc, const void* bias_bf16, void* weight_
   h->map.nout = h->Nout;
   h->map.mode = desc->epi == QL_EPI_SWIGLU ? 1 : 0;
   h->bn = gemm_tile_n(desc->fmt, desc->epi);
-  if (desc->fmt == QL_FP8_E4M3) {
+  if (desc->fmt != QL_NVFP4) {  // FP8 weights (QL_FP8_E4M3, QL_W8A16)
     h->wscale = reinterpret_cast<float*>(h->ws + L.scales);
   } else {
     h->wsf = h->ws + L.scales;
@@ -356,10 +362,14 @@ ql_status finish_create(qlinear_s* h, cudaError_t e, const void* bias_bf16, cuda
     return QL_ERR_CUDA;
   }
   const uint64_t kbytes = h->d.fmt == QL_NVFP4 ? h->K / 2 : h->K;
-  bool ok = make_tmap(&h->tmB1, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, 128,
-                      h->bn, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            make_tmap(&h->tmB2, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, 128,
-                      h->bn / 2, CU_TENSOR_MAP_SWIZZLE_128B);
+  // W8A16: 64 weights per stage land unswizzled for the converter warps
+  const bool w16 = h->d.fmt == QL_W8A16;
+  const uint32_t box = w16 ? 64 : 128;
+  const CUtensorMapSwizzle sw = w16 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B;
+  bool ok = make_tmap(&h->tmB1, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, box,
+                      h->bn, sw) &&
+            make_tmap(&h->tmB2, CU_TENSOR_MAP_DATA_TYPE_UINT8, h->wcodes, kbytes, h->N, kbytes, box,
+                      h->bn / 2, sw);
   if (ok && h->d.fmt == QL_NVFP4)
     ok = make_sf_tmap(&h->tmSFB, h->wsf, sfb_bytes(h->N, h->K, h->bn), 8);
   if (!ok) {
@@ -407,7 +417,7 @@ ql_status qlinear_create(const ql_desc* desc, const void* w_bf16, const void* bi
   if (s != QL_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(h->ws, 0, 1024, st);
-  if (e == cudaSuccess && desc->fmt == QL_FP8_E4M3) {
+  if (e == cudaSuccess && desc->fmt != QL_NVFP4) {
     e = launch_quant_fp8_rows(w_bf16, h->N, h->K, h->K, h->wcodes, h->wscale, h->map, h->num_sms,
                               st);
   } else if (e == cudaSuccess) {
@@ -470,7 +480,12 @@ ql_status qlinear_quantize_act(qlinear_t h, const void* x_bf16, int64_t M, void*
   if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scales)) return QL_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (h->d.fmt == QL_FP8_E4M3) {
+  if (h->d.fmt == QL_W8A16) {
+    // weight-only quantization: the activations stay bf16 (forward may also
+    // be given x itself as `codes`)
+    e = cudaMemcpyAsync(codes, x_bf16, static_cast<size_t>(M) * h->K * 2, cudaMemcpyDeviceToDevice,
+                        st);
+  } else if (h->d.fmt == QL_FP8_E4M3) {
     e = launch_quant_fp8_rows(x_bf16, M, h->K, h->K, static_cast<uint8_t*>(codes),
                               static_cast<float*>(scales), RowMap{0, 0}, h->num_sms, st);
   } else {

@@ -18,7 +18,7 @@ from .tensors import draw
 
 @dataclass(frozen=True)
 class Layer:
-    fmt: str                 # "fp8" | "nvfp4"
+    fmt: str                 # "fp8" | "nvfp4" | "w8a16" (bf16 activations, FP8 weights)
     M: int
     K: int
     N: int                   # GEMM output columns (SwiGLU: gate|up = 2*Nout)
@@ -65,6 +65,9 @@ WORKLOADS = {
         Layer("fp8", 4608, 3072, 9216, "qkv_norm_rope", _N01_OUT8),
     ), "FLUX-dev QKV projection, FP8, 4608x3072x9216, q/k RMS norm per 128-column head + "
        "rotary embedding, v bias"),
+    "flux_qkv_w8a16": Workload("flux_qkv_w8a16", (
+        Layer("w8a16", 4608, 3072, 9216, "bias", _N01_OUT8),
+    ), "FLUX-dev QKV projection, weight-only: bf16 activations x FP8 weights, 4608x3072x9216, bias"),
     "flux_mlp_fp8": Workload("flux_mlp_fp8", (
         Layer("fp8", 4608, 3072, 12288, "bias_gelu", _N01_OUT8),
         Layer("fp8", 4608, 12288, 3072, "bias_gated_residual", _N01, chained=True),

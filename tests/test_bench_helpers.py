@@ -18,3 +18,12 @@ def test_quant_bytes_nvfp4_counts_the_amax_pass():
 def test_weak_scaling_counts_every_rank_over_the_slowest():
     # 2 ranks x 10 steps x 1e12 FLOP in 4 s (the max over ranks) = 5 TFLOP/s
     assert abs(bench.weak_scaling_tflops(1e12, 2, 10, 4000.0) - 5.0) < 1e-12
+
+
+def test_cpu_baseline_runs_for_every_format_and_epilogue():
+    # the oracle leg of the benchmark handles each layer format (and the QKV
+    # epilogue's extra inputs); token counts shrunk so it runs in seconds
+    for name in ("tiny_fp8", "flux2k_swiglu_nvfp4", "flux_qkv_w8a16", "flux_qkv_normrope_fp8"):
+        wl = bench.with_tokens(WORKLOADS[name], 8)
+        tflops, rows, dt, cores = bench.cpu_baseline(wl, 0.01)
+        assert tflops > 0 and 1 <= rows <= 8 and cores >= 1
