@@ -78,7 +78,8 @@ struct Cfg {
   // (B8) and converter warps expand it to bf16 in the MMA's B layout.
   static constexpr bool W16 = (FMT == 2);
   static constexpr bool PAIR = (CG == 2);
-  static constexpr int THREADS = W16 ? 384 : 320;
+  static constexpr int CONV_WARPS = W16 ? 2 : 0;  // FMT 2: weight-stage converters
+  static constexpr int THREADS = 320 + 32 * CONV_WARPS;
   // Tile N: 256, except NVFP4 without SwiGLU, where 224 lets two fp32
   // accumulators (2 x 224 TMEM columns) and the 48 scale-factor columns fit
   // in the 512 columns side by side.
@@ -276,7 +277,7 @@ __global__ void __launch_bounds__(FMT == 2 ? 384 : 320, 1) qgemm_kernel(const __
     mbar_init(smem_u32(&sb->ovl_free), C::EPI_ARRIVALS);
     for (int s = 0; s < 8; ++s) {
       mbar_init(smem_u32(&sb->b8_full[s]), 1);
-      mbar_init(smem_u32(&sb->conv_done[s]), 2 * CG);
+      mbar_init(smem_u32(&sb->conv_done[s]), C::CONV_WARPS * CG);
     }
     mbar_init(smem_u32(&sb->drain), 1);
     sb->abort_flag = 0;
@@ -526,12 +527,18 @@ __global__ void __launch_bounds__(FMT == 2 ? 384 : 320, 1) qgemm_kernel(const __
     }
   } else if (warp >= 2 + NUM_EPI_WARPS) {
     // ------------------------ FMT 2: FP8 weight stage -> bf16 MMA operand
-    // Two warps per CTA.  Row r of this CTA's BN/CG weight rows: 64 E4M3
-    // bytes at B8 + 64 r become 64 bf16 (exact) in the 128-byte-swizzled
-    // K-major layout the MMA descriptor reads: 16-byte chunk c of row r at
-    // B + 128 r + ((c ^ (r & 7)) << 4) (the B region is 1024-byte aligned).
+    // Two warps per CTA.  Each lane takes 16-byte chunks (16 E4M3 codes) of
+    // the raw stage -- consecutive lanes read consecutive chunks, so the
+    // shared loads are contiguous -- and writes them as 32 bytes of bf16
+    // (exact) in the 128-byte-swizzled K-major layout the MMA descriptor
+    // reads: 16-byte chunk c of row r at B + 128 r + ((c ^ (r & 7)) << 4)
+    // (the B region is 1024-byte aligned).  Loads are issued in batches of 8
+    // chunks before any of them is converted.
     if constexpr (C::W16) {
-      const int ct = threadIdx.x - 32 * (2 + NUM_EPI_WARPS);  // 0..63
+      constexpr int NCH = (BN / CG) * 4;                 // raw 16-byte chunks per stage
+      constexpr int PER = NCH / (32 * C::CONV_WARPS);    // per lane: 8 (pair) or 16
+      constexpr int BATCH = PER < 8 ? PER : 8;
+      const int ct = threadIdx.x - 32 * (2 + NUM_EPI_WARPS);  // 0 .. 32 * CONV_WARPS - 1
       const uint32_t done_l0 = mapa_shared(smem_u32(&sb->conv_done[0]), 0);
       int stage = 0;
       uint32_t phase = 0;
@@ -543,21 +550,25 @@ __global__ void __launch_bounds__(FMT == 2 ? 384 : 320, 1) qgemm_kernel(const __
             break;
           }
           uint8_t* st = smem + stage * C::STAGE_BYTES;
-          const uint8_t* b8 = st + A_BYTES + C::B_BYTES;
+          const uint4* b8 = reinterpret_cast<const uint4*>(st + A_BYTES + C::B_BYTES);
           uint8_t* bb = st + A_BYTES;
 #pragma unroll
-          for (int rr = 0; rr < (BN / CG) / 64; ++rr) {
-            const int r = ct + 64 * rr;
+          for (int i0 = 0; i0 < PER; i0 += BATCH) {
+          uint4 c[BATCH];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint4 c = *reinterpret_cast<const uint4*>(b8 + 64 * r + 16 * j);
-              const uint4 lo = make_uint4(e4m3x2_to_bf16x2(c.x), e4m3x2_to_bf16x2(c.x >> 16),
-                                          e4m3x2_to_bf16x2(c.y), e4m3x2_to_bf16x2(c.y >> 16));
-              const uint4 hi = make_uint4(e4m3x2_to_bf16x2(c.z), e4m3x2_to_bf16x2(c.z >> 16),
-                                          e4m3x2_to_bf16x2(c.w), e4m3x2_to_bf16x2(c.w >> 16));
-              *reinterpret_cast<uint4*>(bb + 128 * r + (((2 * j) ^ (r & 7)) << 4)) = lo;
-              *reinterpret_cast<uint4*>(bb + 128 * r + (((2 * j + 1) ^ (r & 7)) << 4)) = hi;
-            }
+          for (int i = 0; i < BATCH; ++i) c[i] = b8[ct + 32 * C::CONV_WARPS * (i0 + i)];
+#pragma unroll
+          for (int i = 0; i < BATCH; ++i) {
+            const int q = ct + 32 * C::CONV_WARPS * (i0 + i);  // raw chunk: row q / 4, chunk q % 4
+            const int r = q >> 2, j = q & 3;
+            uint4 lo, hi;  // elements 0-7, 8-15 of the chunk as bf16
+            e4m3x4_to_bf16x4(c[i].x, lo.x, lo.y);
+            e4m3x4_to_bf16x4(c[i].y, lo.z, lo.w);
+            e4m3x4_to_bf16x4(c[i].z, hi.x, hi.y);
+            e4m3x4_to_bf16x4(c[i].w, hi.z, hi.w);
+            *reinterpret_cast<uint4*>(bb + 128 * r + (((2 * j) ^ (r & 7)) << 4)) = lo;
+            *reinterpret_cast<uint4*>(bb + 128 * r + (((2 * j + 1) ^ (r & 7)) << 4)) = hi;
+          }
           }
           fence_proxy_async_smem();  // generic-proxy writes -> the tensor core's reads
           __syncwarp();

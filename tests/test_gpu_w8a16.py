@@ -62,3 +62,31 @@ def test_w8a16_forward_takes_the_activations_directly():
     _abi.qlinear_forward(lay.h, x.data_ptr(), None, M, None, None, o2.data_ptr(), 0)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2)
+
+
+def test_w8a16_weight_expansion_is_exact_for_every_code():
+    # weight row n holds code (n + k) mod 256 at position k (NaN codes -> 0),
+    # unit scales; activation row m is one-hot at k = 4 m, so out[m, n] must be
+    # the E4M3 value of code (n + 4 m) mod 256 bit for bit (every E4M3 value,
+    # subnormals included, is a bf16 value) -- for every code and for 16
+    # positions spread over the 16-byte chunks of a stage
+    import torch
+    import precision_gemm_qlinear_b200 as ql
+    N, K, M = 256, 64, 16
+    codes = ((np.arange(N)[:, None] + np.arange(K)[None, :]) % 256).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0
+    x = np.zeros((M, K), np.uint16)
+    x[np.arange(M), 4 * np.arange(M)] = 0x3F80  # 1.0
+    lay = ql.QLinear.from_quantized("w8a16", "bias", torch.from_numpy(codes).cuda(),
+                                    torch.ones(N, dtype=torch.float32, device="cuda"))
+    out = lay(to_dev_bf16(x))
+    torch.cuda.synchronize()
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    dec = np.array([oracle.e4m3_decode(c) for c in range(256)], np.float32)
+    sel = codes[:, 4 * np.arange(M)].T
+    want = (dec[sel].view(np.uint32) >> 16).astype(np.uint16)
+    # code 0x80 is -0: summed with the +0 products of the other positions it
+    # is +0, as IEEE addition gives
+    want[sel == 0x80] = 0
+    bad = sorted({int(c) for c in sel[got != want]})
+    assert not bad, f"E4M3 codes expanded wrongly: {bad}"
