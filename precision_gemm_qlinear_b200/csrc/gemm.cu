@@ -207,22 +207,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* p, float (&o)[32]) {
-  const uint4* q = reinterpret_cast<const uint4*>(p);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint4 v = __ldg(q + i);
-    o[8 * i + 0] = bf16lo(v.x);
-    o[8 * i + 1] = bf16hi(v.x);
-    o[8 * i + 2] = bf16lo(v.y);
-    o[8 * i + 3] = bf16hi(v.y);
-    o[8 * i + 4] = bf16lo(v.z);
-    o[8 * i + 5] = bf16hi(v.z);
-    o[8 * i + 6] = bf16lo(v.w);
-    o[8 * i + 7] = bf16hi(v.w);
-  }
-}
-
 // 32 bf16 kept packed (16 registers); element i is bf16x32_at(v, i).
 __device__ __forceinline__ void load_bf16x32_packed(const __nv_bfloat16* p, uint4 (&v)[4]) {
   const uint4* q = reinterpret_cast<const uint4*>(p);
