@@ -38,7 +38,7 @@ L2_BYTES = 126 * 2 ** 20
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # nominal dense tensor-core ratios to bf16 (FP8 4.5 / 2.25 PF, FP4 9 / 2.25 PF)
 NOMINAL_RATIO = {"fp8": 2.0, "nvfp4": 4.0, "w8a16": 1.0}  # w8a16 runs bf16 MMAs
-GEMM_SOURCES = ["precision_gemm_qlinear_b200/csrc/gemm.cu",
+GEMM_SOURCES = ["precision_gemm_qlinear_b200/csrc/gemm.cu", "precision_gemm_qlinear_b200/csrc/codec.cuh",
                 "precision_gemm_qlinear_b200/csrc/ptx.cuh",
                 "precision_gemm_qlinear_b200/csrc/internal.h"]
 
