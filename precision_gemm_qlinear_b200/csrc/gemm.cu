@@ -45,9 +45,7 @@ namespace {
 
 constexpr int BM = 128;                // rows of the tile per CTA
 constexpr int BK_BYTES = 128;          // K bytes per pipeline stage
-constexpr int A_BYTES = BM * BK_BYTES;  // 16 KB
-constexpr int NUM_EPI_WARPS = 8;
-constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+constexpr int A_TILE_BYTES = BM * BK_BYTES;  // one 128-row A box: 16 KB
 constexpr int STAGING_BYTES = 32 * 64;  // one 32 x 32 bf16 box
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;  // 1 s
 
@@ -78,12 +76,23 @@ struct Cfg {
   // (B8) and converter warps expand it to bf16 in the MMA's B layout.
   static constexpr bool W16 = (FMT == 2);
   static constexpr bool PAIR = (CG == 2);
-  static constexpr int CONV_WARPS = W16 ? 2 : 0;  // FMT 2: weight-stage converters
-  static constexpr int THREADS = 320 + 32 * CONV_WARPS;
+  // Warps: producer, MMA, epilogue, and for FMT 2 the weight-stage
+  // converters.  FMT 2 tiles take long enough in the main loop that four
+  // epilogue warps (two passes each, over the halves eight warps would
+  // share) keep up, which leaves room for four converters at 320 threads.
+  static constexpr int EPI_WARPS = W16 ? 4 : 8;
+  static constexpr int EPI_PASSES = 8 / EPI_WARPS;
+  static constexpr int CONV_WARPS = W16 ? 4 : 0;
+  static constexpr int THREADS = 64 + 32 * (EPI_WARPS + CONV_WARPS);
   // Tile N: 256, except NVFP4 without SwiGLU, where 224 lets two fp32
   // accumulators (2 x 224 TMEM columns) and the 48 scale-factor columns fit
   // in the 512 columns side by side.
-  static constexpr int BN = (NV && EPI != EPI_SWIGLU && EPI != EPI_QKV) ? 224 : 256;
+  // FMT 2 with an epilogue that does not need 256-column tiles: each CTA
+  // computes MSUB = 2 row subtiles against the same converted weight stage
+  // (tile (2 x 128 CG) x 128), halving the conversion per MMA.
+  static constexpr int MSUB = (FMT == 2 && EPI != EPI_SWIGLU && EPI != EPI_QKV) ? 2 : 1;
+  static constexpr int BN = (NV && EPI != EPI_SWIGLU && EPI != EPI_QKV) ? 224 : (MSUB == 2 ? 128 : 256);
+  static constexpr int A_BYTES = MSUB * A_TILE_BYTES;  // this stage's rows of A
   static constexpr int B_BYTES = (BN / CG) * BK_BYTES;  // this CTA's rows of B
   static constexpr int SFA_BYTES = NV ? 2048 : 0;       // 4 atoms (one per MMA K step)
   static constexpr int SFB_BYTES = NV ? 16384 : 0;      // 4 replicated 4 KB chunks (all 256 B rows)
@@ -92,9 +101,9 @@ struct Cfg {
   static constexpr int STAGES = NV ? (PAIR ? 4 : 3) : (W16 ? (PAIR ? 4 : 3) : (PAIR ? 6 : 4));
   // staging buffers per epilogue warp: two unless that breaks the budget
   static constexpr int NBUF =
-      (STAGES * STAGE_BYTES + NUM_EPI_WARPS * 2 * STAGING_BYTES + 512 + 1024 <= 232448) ? 2 : 1;
+      (STAGES * STAGE_BYTES + EPI_WARPS * 2 * STAGING_BYTES + 512 + 1024 <= 232448) ? 2 : 1;
   static constexpr int STAGING_OFF = STAGES * STAGE_BYTES;
-  static constexpr int BAR_OFF = STAGING_OFF + NUM_EPI_WARPS * NBUF * STAGING_BYTES;
+  static constexpr int BAR_OFF = STAGING_OFF + EPI_WARPS * NBUF * STAGING_BYTES;
   static_assert(BAR_OFF + 512 + 1024 <= 232448, "shared memory budget");
   static constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;  // + barriers + alignment slack
   // TMEM columns: FP8 -> two disjoint 256-column accumulators.  NVFP4 ->
@@ -104,11 +113,12 @@ struct Cfg {
   // [0,256) and [192,448), overlapping in [192,256), and the epilogue reads
   // the shared columns first and releases them early.
   static constexpr bool OVL = NV && BN == 256;
-  static constexpr uint32_t ACC1 = OVL ? 192 : BN;
+  static constexpr uint32_t ACC1 = OVL ? 192 : MSUB * BN;
   static constexpr uint32_t SFA_COL = 448;
   static constexpr uint32_t SFB_COL = 464;
   static_assert(!NV || ACC1 + BN <= SFA_COL, "TMEM budget");
-  static constexpr uint32_t EPI_ARRIVALS = NUM_EPI_WARPS * CG;  // per tile, at the leader
+  // per tile, at the leader: one per epilogue warp and pass
+  static constexpr uint32_t EPI_ARRIVALS = EPI_WARPS * EPI_PASSES * CG;
 };
 
 struct SmemBars {
@@ -235,7 +245,8 @@ __device__ __forceinline__ void load_f32x32(const float* p, float (&o)[32]) {
 // OQ = 1: the epilogue writes NVFP4 codes and block scales for the next
 // layer instead of bf16 (see GemmParams::q_*).
 template <int FMT, int EPI, int CG, int OQ>
-__global__ void __launch_bounds__(FMT == 2 ? 384 : 320, 1) qgemm_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
+    qgemm_kernel(const __grid_constant__ GemmParams p) {
   using C = Cfg<FMT, CG, EPI>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
@@ -261,7 +272,7 @@ __global__ void __launch_bounds__(FMT == 2 ? 384 : 320, 1) qgemm_kernel(const __
     mbar_init(smem_u32(&sb->ovl_free), C::EPI_ARRIVALS);
     for (int s = 0; s < 8; ++s) {
       mbar_init(smem_u32(&sb->b8_full[s]), 1);
-      mbar_init(smem_u32(&sb->conv_done[s]), C::CONV_WARPS * CG);
+      mbar_init(smem_u32(&sb->conv_done[s]), CG);  // one converter warp per CTA
     }
     mbar_init(smem_u32(&sb->drain), 1);
     sb->abort_flag = 0;
@@ -301,7 +312,7 @@ __global__ void __launch_bounds__(FMT == 2 ? 384 : 320, 1) qgemm_kernel(const __
       for (int t = unit; t < num_tiles && ok; t += nunits) {
         int mb, nb;
         tile_coords(t, p, mb, nb);
-        const int a_row = mb * (BM * CG) + static_cast<int>(rank) * BM;
+        const int a_row = mb * (BM * CG * C::MSUB) + static_cast<int>(rank) * BM;  // subtile 0
         const int b_row = nb * BN + static_cast<int>(rank) * (BN / CG);
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!wait_bar(&sb->empty[stage], phase ^ 1, sb, p.err, ERR_WAIT_PRODUCER)) {
@@ -322,22 +333,25 @@ __global__ void __launch_bounds__(FMT == 2 ? 384 : 320, 1) qgemm_kernel(const __
                 // bf16 activations (64 elements = 128 bytes per stage) counted
                 // at the leader; the raw FP8 weights on this CTA's own barrier,
                 // where this CTA's converter warps wait for them
-                if (rank == 0) mbar_arrive_expect_tx(fb, 2 * A_BYTES);
-                tma_load_2d_pair(smem_u32(st), &p.tmA, lfb, kb * 64, a_row);
+                if (rank == 0) mbar_arrive_expect_tx(fb, 2 * C::A_BYTES);
+#pragma unroll
+                for (int sub = 0; sub < C::MSUB; ++sub)
+                  tma_load_2d_pair(smem_u32(st + sub * A_TILE_BYTES), &p.tmA, lfb, kb * 64,
+                                   a_row + sub * BM * CG);
                 const uint32_t xb = smem_u32(&sb->b8_full[stage]);
                 mbar_arrive_expect_tx(xb, C::B8_BYTES);
-                tma_load_2d(smem_u32(st + A_BYTES + C::B_BYTES), &p.tmB, xb, kb * 64, b_row);
+                tma_load_2d(smem_u32(st + C::A_BYTES + C::B_BYTES), &p.tmB, xb, kb * 64, b_row);
               } else {
               if (rank == 0) mbar_arrive_expect_tx(fb, 2 * C::STAGE_BYTES);
               tma_load_2d_pair(smem_u32(st), &p.tmA, lfb, kb * BK_BYTES, a_row);
-              tma_load_2d_pair(smem_u32(st + A_BYTES), &p.tmB, lfb, kb * BK_BYTES, b_row);
+              tma_load_2d_pair(smem_u32(st + C::A_BYTES), &p.tmB, lfb, kb * BK_BYTES, b_row);
               }
               if constexpr (C::NV) {
                 // scales through 2-D maps of 2048-byte rows (uint64 x 256): the
                 // A atoms of this CTA's 128 rows (one row of the map) and the
                 // replicated B chunks of all 256 columns of the tile (8 rows;
                 // both CTAs need them)
-                const uint32_t sfs = smem_u32(st + A_BYTES + C::B_BYTES);
+                const uint32_t sfs = smem_u32(st + C::A_BYTES + C::B_BYTES);
                 const int ka = p.sf_kchunks_a >> 2;
                 tma_load_2d_pair(sfs, &p.tmSFA, lfb, 0, (mb * 2 + static_cast<int>(rank)) * ka + kb);
                 tma_load_2d_pair(sfs + C::SFA_BYTES, &p.tmSFB, lfb, 0,
@@ -345,22 +359,25 @@ __global__ void __launch_bounds__(FMT == 2 ? 384 : 320, 1) qgemm_kernel(const __
               }
             } else {
               if constexpr (C::W16) {
-                mbar_arrive_expect_tx(fb, A_BYTES);
-                tma_load_2d(smem_u32(st), &p.tmA, fb, kb * 64, a_row);
+                mbar_arrive_expect_tx(fb, C::A_BYTES);
+#pragma unroll
+                for (int sub = 0; sub < C::MSUB; ++sub)
+                  tma_load_2d(smem_u32(st + sub * A_TILE_BYTES), &p.tmA, fb, kb * 64,
+                              a_row + sub * BM * CG);
                 const uint32_t xb = smem_u32(&sb->b8_full[stage]);
                 mbar_arrive_expect_tx(xb, C::B8_BYTES);
-                tma_load_2d(smem_u32(st + A_BYTES + C::B_BYTES), &p.tmB, xb, kb * 64, b_row);
+                tma_load_2d(smem_u32(st + C::A_BYTES + C::B_BYTES), &p.tmB, xb, kb * 64, b_row);
               } else {
               mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
               tma_load_2d(smem_u32(st), &p.tmA, fb, kb * BK_BYTES, a_row);
-              tma_load_2d(smem_u32(st + A_BYTES), &p.tmB, fb, kb * BK_BYTES, b_row);
+              tma_load_2d(smem_u32(st + C::A_BYTES), &p.tmB, fb, kb * BK_BYTES, b_row);
               }
               if constexpr (C::NV) {
                 const uint8_t* sfa =
                     p.sfa + (static_cast<int64_t>(mb) * p.sf_kchunks_a + kb * 4) * 512;
                 const uint8_t* sfb =
                     p.sfb + (static_cast<int64_t>(nb) * p.sfb_nstages + kb) * C::SFB_BYTES;
-                const uint32_t sfs = smem_u32(st + A_BYTES + C::B_BYTES);
+                const uint32_t sfs = smem_u32(st + C::A_BYTES + C::B_BYTES);
                 bulk_load(sfs, sfa, C::SFA_BYTES, fb);
                 bulk_load(sfs + C::SFA_BYTES, sfb, C::SFB_BYTES, fb);
               }
@@ -409,9 +426,10 @@ __global__ void __launch_bounds__(FMT == 2 ? 384 : 320, 1) qgemm_kernel(const __
       // stage-0 operand and scale descriptors, scale-factor TMEM addresses.
       const uint32_t s0 = smem_u32(smem);
       const uint64_t d_a0 = sdesc_k_sw128(s0);
-      const uint64_t d_b0 = sdesc_k_sw128(s0 + A_BYTES);
-      const uint64_t d_sfa0 = sdesc_k_interleave(s0 + A_BYTES + C::B_BYTES);
-      const uint64_t d_sfb0 = sdesc_k_interleave2(s0 + A_BYTES + C::B_BYTES + C::SFA_BYTES, 128, 256);
+      const uint64_t d_b0 = sdesc_k_sw128(s0 + C::A_BYTES);
+      const uint64_t d_sfa0 = sdesc_k_interleave(s0 + C::A_BYTES + C::B_BYTES);
+      const uint64_t d_sfb0 =
+          sdesc_k_interleave2(s0 + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, 128, 256);
       const uint32_t t_sfa = tmem + C::SFA_COL;
       const uint32_t t_sfb = tmem + C::SFB_COL;
       for (int t = unit; t < num_tiles && ok; t += nunits, ++local) {
@@ -470,10 +488,15 @@ __global__ void __launch_bounds__(FMT == 2 ? 384 : 320, 1) qgemm_kernel(const __
                 mma_mxf4nvf4(d_tmem, ad, bd, idesc_f4<CG, BN>(), t_sfa + 4 * j, t_sfb + 8 * j,
                              acc);
             } else if constexpr (C::W16) {
-              if constexpr (C::PAIR)
-                mma_bf16_pair(d_tmem, ad, bd, idesc_bf16<CG, BN>(), acc);
-              else
-                mma_bf16(d_tmem, ad, bd, idesc_bf16<CG, BN>(), acc);
+              // one MMA per row subtile, all against the same B stage
+#pragma unroll
+              for (int sub = 0; sub < C::MSUB; ++sub) {
+                const uint64_t as = ad + sub * (A_TILE_BYTES >> 4);
+                if constexpr (C::PAIR)
+                  mma_bf16_pair(d_tmem + sub * BN, as, bd, idesc_bf16<CG, BN>(), acc);
+                else
+                  mma_bf16(d_tmem + sub * BN, as, bd, idesc_bf16<CG, BN>(), acc);
+              }
             } else {
               if constexpr (C::PAIR)
                 mma_f8f6f4_pair(d_tmem, ad, bd, idesc_f8<CG, BN>(), acc);
@@ -509,41 +532,55 @@ __global__ void __launch_bounds__(FMT == 2 ? 384 : 320, 1) qgemm_kernel(const __
         }
       }
     }
-  } else if (warp >= 2 + NUM_EPI_WARPS) {
+  } else if (warp >= 2 + C::EPI_WARPS) {
     // ------------------------ FMT 2: FP8 weight stage -> bf16 MMA operand
-    // Two warps per CTA.  Each lane takes 16-byte chunks (16 E4M3 codes) of
-    // the raw stage -- consecutive lanes read consecutive chunks, so the
-    // shared loads are contiguous -- and writes them as 32 bytes of bf16
-    // (exact) in the 128-byte-swizzled K-major layout the MMA descriptor
-    // reads: 16-byte chunk c of row r at B + 128 r + ((c ^ (r & 7)) << 4)
-    // (the B region is 1024-byte aligned).  Loads are issued in batches of 8
-    // chunks before any of them is converted.
+    // Four warps per CTA, each owning the stages s with s % 4 == its index
+    // (with three stages the fourth warp has none): a warp converts a whole
+    // stage, so the fence that publishes one stage to the tensor core
+    // overlaps the other warps' conversion of the next ones.  Owning whole
+    // stages keeps every warp's waits on a stage's barrier in the order of
+    // its phases (a parity wait must never run two phases ahead).  Each lane takes
+    // 16-byte chunks (16 E4M3 codes) of the raw stage -- consecutive lanes
+    // read consecutive chunks, so the shared loads are contiguous -- and
+    // writes them as 32 bytes of bf16 (exact) in the 128-byte-swizzled
+    // K-major layout the MMA descriptor reads: 16-byte chunk c of row r at
+    // B + 128 r + ((c ^ (r & 7)) << 4) (the B region is 1024-byte aligned).
+    // Loads are issued in batches of 8 chunks before any of them is
+    // converted.
     if constexpr (C::W16) {
-      constexpr int NCH = (BN / CG) * 4;                 // raw 16-byte chunks per stage
-      constexpr int PER = NCH / (32 * C::CONV_WARPS);    // per lane: 8 (pair) or 16
+      constexpr int NCH = (BN / CG) * 4;  // raw 16-byte chunks per stage
+      constexpr int PER = NCH / 32;       // per lane: 8 or 16 (pair), 16 or 32 (one CTA)
       constexpr int BATCH = PER < 8 ? PER : 8;
-      const int ct = threadIdx.x - 32 * (2 + NUM_EPI_WARPS);  // 0 .. 32 * CONV_WARPS - 1
+      const int ct = lane;
+      const int cw = warp - (2 + C::EPI_WARPS);  // converter warp: 0 .. CONV_WARPS - 1
       const uint32_t done_l0 = mapa_shared(smem_u32(&sb->conv_done[0]), 0);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int t = unit; t < num_tiles && ok; t += nunits) {
         for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (stage % C::CONV_WARPS != cw) {
+            if (++stage == C::STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
+            continue;
+          }
           if (!wait_bar(&sb->b8_full[stage], phase, sb, p.err, ERR_WAIT_EPI)) {
             ok = false;
             break;
           }
           uint8_t* st = smem + stage * C::STAGE_BYTES;
-          const uint4* b8 = reinterpret_cast<const uint4*>(st + A_BYTES + C::B_BYTES);
-          uint8_t* bb = st + A_BYTES;
+          const uint4* b8 = reinterpret_cast<const uint4*>(st + C::A_BYTES + C::B_BYTES);
+          uint8_t* bb = st + C::A_BYTES;
 #pragma unroll
           for (int i0 = 0; i0 < PER; i0 += BATCH) {
           uint4 c[BATCH];
 #pragma unroll
-          for (int i = 0; i < BATCH; ++i) c[i] = b8[ct + 32 * C::CONV_WARPS * (i0 + i)];
+          for (int i = 0; i < BATCH; ++i) c[i] = b8[ct + 32 * (i0 + i)];
 #pragma unroll
           for (int i = 0; i < BATCH; ++i) {
-            const int q = ct + 32 * C::CONV_WARPS * (i0 + i);  // raw chunk: row q / 4, chunk q % 4
+            const int q = ct + 32 * (i0 + i);  // raw chunk: row q / 4, chunk q % 4
             const int r = q >> 2, j = q & 3;
             uint4 lo, hi;  // elements 0-7, 8-15 of the chunk as bf16
             e4m3x4_to_bf16x4(c[i].x, lo.x, lo.y);
@@ -566,13 +603,12 @@ __global__ void __launch_bounds__(FMT == 2 ? 384 : 320, 1) qgemm_kernel(const __
     }
   } else {
     // --------------------------------------------------------- epilogue
-    const int ew = warp - 2;           // 0..7
+    const int ew = warp - 2;           // 0 .. EPI_WARPS - 1
     const int sp = warp & 3;           // TMEM sub-partition: rows [32 sp, 32 sp + 32) of the CTA tile
-    const int half = ew >> 2;          // the two warps of a sub-partition take alternate chunks
     uint8_t* staging = smem + C::STAGING_OFF + ew * C::NBUF * STAGING_BYTES;
-    // 32-column output chunks per tile, and this warp's share of them
+    // 32-column output chunks per tile
     constexpr int NCHT = (EPI == EPI_SWIGLU) ? BN / 64 : BN / 32;
-    const int nch = (NCHT - half + 1) >> 1;
+    constexpr bool MS = C::MSUB == 2;
     const uint32_t ovl_l0 = mapa_shared(smem_u32(&sb->ovl_free), 0);
     int local = 0;
     uint32_t nstore = 0;
@@ -592,282 +628,296 @@ __global__ void __launch_bounds__(FMT == 2 ? 384 : 320, 1) qgemm_kernel(const __
       const uint32_t use = static_cast<uint32_t>(local >> 1);
       if (!wait_bar(&sb->acc_full[buf], use & 1, sb, p.err, ERR_WAIT_EPI)) break;
       tc_fence_after();
-      const int row0 = mb * (BM * CG) + static_cast<int>(rank) * BM + sp * 32;  // first row of this warp
-      const int m = row0 + lane;
-      const bool row_ok = m < p.M;
-      const bool slab_ok = row0 < p.M;
-      float rs;
-      if constexpr (C::NV)
-        rs = __ldg(p.ga) * __ldg(p.gw);
-      else if constexpr (C::W16)
-        rs = 1.f;  // bf16 activations carry no scale
-      else
-        rs = row_ok ? __ldg(p.sa + m) : 0.f;
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(sp * 32) << 16) + (buf ? C::ACC1 : 0u);
-      // one 32 x 32 bf16 box: swizzled shared staging, then a TMA store
-      auto store_chunk = [&](const uint32_t (&pk)[16], int ocol) {
-        uint8_t* sbuf = staging + (nstore % C::NBUF) * STAGING_BYTES;
-        if (lane == 0) bulk_wait_group_read<C::NBUF - 1>();
-        __syncwarp();
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int sw = (j ^ ((lane >> 1) & 3)) << 4;
-          *reinterpret_cast<uint4*>(sbuf + lane * 64 + sw) =
-              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0 && slab_ok) {
-          tma_store_2d(&p.tmC, smem_u32(sbuf), ocol, row0);
-          bulk_commit_group();
-        }
-        ++nstore;
-      };
-      if constexpr (EPI == EPI_QKV) {
-        // One 128-column head per warp (head `half` of the tile).  Pass 1:
-        // the head's sum of squares (q and k heads); pass 2: re-read TMEM,
-        // normalize, weight, rotate the pairs, store.  Both passes recompute
-        // v = acc * scale + bias from TMEM instead of keeping 128 values.
-        const int h0 = nb * BN + QKV_HEAD_DIM * half;
-        const uint32_t hb = tbase + QKV_HEAD_DIM * half;
-        const bool hlive = h0 < p.N;
-        const bool normed = h0 < p.qk_cols;
-        const float* wgt = p.qk_w + (h0 < p.k_col0 ? 0 : QKV_HEAD_DIM);
-        const int64_t mrow = row_ok ? m : p.M - 1;  // padded rows read row M-1's angles
-        auto values = [&](int k, const uint32_t (&a)[32], float (&v)[32]) {
-          uint4 bp[4];
-          load_bf16x32_packed(p.bias + h0 + 32 * k, bp);
-          if constexpr (C::NV) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = fmaf(__uint_as_float(a[i]), rs, bf16x32_at(bp, i));
-          } else {
-            const float4* swp = reinterpret_cast<const float4*>(p.sw + h0 + 32 * k);
-#pragma unroll
-            for (int i4 = 0; i4 < 8; ++i4) {
-              const float4 s4 = __ldg(swp + i4);
-              const float sw4[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int i = 4 * i4 + j;
-                v[i] = fmaf(__uint_as_float(a[i]), rs * sw4[j], bf16x32_at(bp, i));
+      // Each sub-partition's work is split in two halves: with eight
+      // epilogue warps the two warps of a sub-partition take one each, with
+      // four each warp takes both, one per pass.  A half is the row subtile
+      // (two subtiles per CTA), else alternate 32-column chunks (the head,
+      // for QKV).  Every (warp, pass) releases the accumulator once.
+#pragma unroll 1
+      for (int pass = 0; pass < C::EPI_PASSES; ++pass) {
+        const int half = C::EPI_PASSES == 2 ? pass : (ew >> 2);
+        const int nch = MS ? NCHT : (NCHT - half + 1) >> 1;  // this half's chunks
+        const int sub = MS ? half : 0;  // row subtile of this warp
+        const int row0 = mb * (BM * CG * C::MSUB) + sub * (BM * CG) + static_cast<int>(rank) * BM +
+                         sp * 32;  // first row of this warp
+        const int m = row0 + lane;
+        const bool row_ok = m < p.M;
+        const bool slab_ok = row0 < p.M;
+        float rs;
+        if constexpr (C::NV)
+          rs = __ldg(p.ga) * __ldg(p.gw);
+        else if constexpr (C::W16)
+          rs = 1.f;  // bf16 activations carry no scale
+        else
+          rs = row_ok ? __ldg(p.sa + m) : 0.f;
+        const uint32_t tbase = tmem + (static_cast<uint32_t>(sp * 32) << 16) + (buf ? C::ACC1 : 0u) +
+                               static_cast<uint32_t>(sub * BN);
+        // one 32 x 32 bf16 box: swizzled shared staging, then a TMA store
+        auto store_chunk = [&](const uint32_t (&pk)[16], int ocol) {
+          uint8_t* sbuf = staging + (nstore % C::NBUF) * STAGING_BYTES;
+          if (lane == 0) bulk_wait_group_read<C::NBUF - 1>();
+          __syncwarp();
+  #pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int sw = (j ^ ((lane >> 1) & 3)) << 4;
+            *reinterpret_cast<uint4*>(sbuf + lane * 64 + sw) =
+                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && slab_ok) {
+            tma_store_2d(&p.tmC, smem_u32(sbuf), ocol, row0);
+            bulk_commit_group();
+          }
+          ++nstore;
+        };
+        if constexpr (EPI == EPI_QKV) {
+          // One 128-column head per warp (head `half` of the tile).  Pass 1:
+          // the head's sum of squares (q and k heads); pass 2: re-read TMEM,
+          // normalize, weight, rotate the pairs, store.  Both passes recompute
+          // v = acc * scale + bias from TMEM instead of keeping 128 values.
+          const int h0 = nb * BN + QKV_HEAD_DIM * half;
+          const uint32_t hb = tbase + QKV_HEAD_DIM * half;
+          const bool hlive = h0 < p.N;
+          const bool normed = h0 < p.qk_cols;
+          const float* wgt = p.qk_w + (h0 < p.k_col0 ? 0 : QKV_HEAD_DIM);
+          const int64_t mrow = row_ok ? m : p.M - 1;  // padded rows read row M-1's angles
+          auto values = [&](int k, const uint32_t (&a)[32], float (&v)[32]) {
+            uint4 bp[4];
+            load_bf16x32_packed(p.bias + h0 + 32 * k, bp);
+            if constexpr (C::NV) {
+  #pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = fmaf(__uint_as_float(a[i]), rs, bf16x32_at(bp, i));
+            } else {
+              const float4* swp = reinterpret_cast<const float4*>(p.sw + h0 + 32 * k);
+  #pragma unroll
+              for (int i4 = 0; i4 < 8; ++i4) {
+                const float4 s4 = __ldg(swp + i4);
+                const float sw4[4] = {s4.x, s4.y, s4.z, s4.w};
+  #pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const int i = 4 * i4 + j;
+                  v[i] = fmaf(__uint_as_float(a[i]), rs * sw4[j], bf16x32_at(bp, i));
+                }
               }
             }
-          }
-        };
-        if (!hlive) {
-          // a head past N (ragged N tile): nothing to read, release at once
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            if (C::OVL) mbar_arrive_cluster(ovl_l0);
-            mbar_arrive_cluster(mapa_shared(smem_u32(&sb->acc_empty[buf]), 0));
-          }
-          continue;
-        }
-        // steps: 4 sum-of-squares chunks (q, k heads), then the 4 output
-        // chunks; the next step's TMEM load is in flight during each step
-        const int nsteps = normed ? 8 : 4;
-        uint32_t ha[32], hb2[32];
-        tmem_ld_32x32b_x32(hb, ha);
-        float ss = 0.f, rn = 1.f;
-        auto step = [&](int t, const uint32_t (&cur)[32], uint32_t (&nxt)[32]) {
-          const int k = t & 3;
-          tmem_wait_ld();
-          if (t + 1 < nsteps) tmem_ld_32x32b_x32(hb + 32 * ((t + 1) & 3), nxt);
-          if (t == nsteps - 1) {
-            // the whole head has been read: release this warp's share of both
-            // buffers (the overlap columns of NVFP4's 256-wide tiles included)
+          };
+          if (!hlive) {
+            // a head past N (ragged N tile): nothing to read, release at once
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
               if (C::OVL) mbar_arrive_cluster(ovl_l0);
               mbar_arrive_cluster(mapa_shared(smem_u32(&sb->acc_empty[buf]), 0));
             }
+            continue;
           }
-          float v[32];
-          values(k, cur, v);
-          if (normed && t < 4) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
-            if (k == 3) rn = rsqrtf(fmaf(ss, 1.f / QKV_HEAD_DIM, p.qk_eps));
-            return;
-          }
-          if (normed) {
-            const float4* wp = reinterpret_cast<const float4*>(wgt + 32 * k);
-            const float4* cp =
-                reinterpret_cast<const float4*>(p.rope_cos + mrow * (QKV_HEAD_DIM / 2) + 16 * k);
-            const float4* snp =
-                reinterpret_cast<const float4*>(p.rope_sin + mrow * (QKV_HEAD_DIM / 2) + 16 * k);
-#pragma unroll
-            for (int j4 = 0; j4 < 4; ++j4) {
-              const float4 c4 = __ldg(cp + j4), s4 = __ldg(snp + j4);
-              const float4 w0 = __ldg(wp + 2 * j4), w1 = __ldg(wp + 2 * j4 + 1);
-              const float cs[4] = {c4.x, c4.y, c4.z, c4.w}, sn[4] = {s4.x, s4.y, s4.z, s4.w};
-              const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-              for (int tt = 0; tt < 4; ++tt) {
-                const int i = 2 * (4 * j4 + tt);
-                const float x0 = v[i] * rn * wv[2 * tt], x1 = v[i + 1] * rn * wv[2 * tt + 1];
-                v[i] = fmaf(x0, cs[tt], -x1 * sn[tt]);
-                v[i + 1] = fmaf(x0, sn[tt], x1 * cs[tt]);
+          // steps: 4 sum-of-squares chunks (q, k heads), then the 4 output
+          // chunks; the next step's TMEM load is in flight during each step
+          const int nsteps = normed ? 8 : 4;
+          uint32_t ha[32], hb2[32];
+          tmem_ld_32x32b_x32(hb, ha);
+          float ss = 0.f, rn = 1.f;
+          auto step = [&](int t, const uint32_t (&cur)[32], uint32_t (&nxt)[32]) {
+            const int k = t & 3;
+            tmem_wait_ld();
+            if (t + 1 < nsteps) tmem_ld_32x32b_x32(hb + 32 * ((t + 1) & 3), nxt);
+            if (t == nsteps - 1) {
+              // the whole head has been read: release this warp's share of both
+              // buffers (the overlap columns of NVFP4's 256-wide tiles included)
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) {
+                if (C::OVL) mbar_arrive_cluster(ovl_l0);
+                mbar_arrive_cluster(mapa_shared(smem_u32(&sb->acc_empty[buf]), 0));
               }
             }
-          }
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) pk[i >> 1] = pack_bf16x2(v[i], v[i + 1]);
-          store_chunk(pk, h0 + 32 * k);
-        };
-#pragma unroll 1
-        for (int t = 0; t < nsteps; t += 2) {
-          step(t, ha, hb2);
-          step(t + 1, hb2, ha);
-        }
-        continue;
-      }
-      // chunk processed at step ci.  SwiGLU with overlapping buffers: the
-      // shared columns are the up half of output chunks 2, 3 in buffer 0 and
-      // the gate half of chunks 0, 1 in buffer 1; every warp holds exactly one
-      // of them and reads it first.
-      auto chunk_of = [&](int ci) {
-        const int k = (C::OVL && buf == 0) ? (nch - 1 - ci) : ci;
-        return half + 2 * k;
-      };
-      constexpr int NCHW = (NCHT + 1) / 2;  // most chunks a warp can have
-      uint32_t acc[2][32];                   // double-buffered accumulator chunk
-      uint32_t accu[32];                     // SwiGLU: the up half
-      tmem_ld_32x32b_x32(tbase + 32 * chunk_of(0), acc[0]);
-      if constexpr (EPI == EPI_SWIGLU) tmem_ld_32x32b_x32(tbase + 128 + 32 * chunk_of(0), accu);
-#pragma unroll
-      for (int ci = 0; ci < NCHW; ++ci) {
-        if (ci >= nch) break;
-        const int c = chunk_of(ci);
-        const int ncol = nb * BN + 32 * c;                                     // GEMM column of acc[..][0]
-        const int ocol = (EPI == EPI_SWIGLU) ? nb * (BN / 2) + 32 * c : ncol;  // output column
-        // SwiGLU (N = 256): gate columns ncol.., up columns ncol + 128..
-        const bool live = ncol < p.N;  // past the last column (N % 32 == 0); warp-uniform
-        // per-column and per-row operands: issued before the TMEM wait so the
-        // two latencies overlap
-        uint4 bias_a[4], bias_b[4], gate_a[4], res_a[4];
-        float sw_a[32];
-        if (live) {
-          load_bf16x32_packed(p.bias + ncol, bias_a);
-          if constexpr (!C::NV) load_f32x32(p.sw + ncol, sw_a);
-          if constexpr (EPI == EPI_SWIGLU) {
-            load_bf16x32_packed(p.bias + ncol + 128, bias_b);
-          }
-          if constexpr (EPI == EPI_GATED_RES) {
-            // per-batch gates (CFG-batched tokens): row m uses gate row m / gate_rows
-            const __nv_bfloat16* gp = p.gate + ocol;
-            if (p.gate_rows > 0)
-              gp += static_cast<int64_t>((row_ok ? m : p.M - 1) / p.gate_rows) * p.Nout;
-            load_bf16x32_packed(gp, gate_a);
-            if (row_ok) {
-              load_bf16x32_packed(p.residual + static_cast<int64_t>(m) * p.Nout + ocol, res_a);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) res_a[i] = make_uint4(0u, 0u, 0u, 0u);
+            float v[32];
+            values(k, cur, v);
+            if (normed && t < 4) {
+  #pragma unroll
+              for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
+              if (k == 3) rn = rsqrtf(fmaf(ss, 1.f / QKV_HEAD_DIM, p.qk_eps));
+              return;
             }
-          }
-        }
-        tmem_wait_ld();
-        // the next chunk's accumulators stream in while this one is computed
-        if constexpr (EPI != EPI_SWIGLU) {
-          if (ci + 1 < nch) tmem_ld_32x32b_x32(tbase + 32 * chunk_of(ci + 1), acc[(ci + 1) & 1]);
-        }
-        if (C::OVL && ci == 0) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(ovl_l0);
-        }
-        if (ci == nch - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sb->acc_empty[buf]), 0));
-        }
-        const uint32_t* ra = acc[(EPI == EPI_SWIGLU) ? 0 : (ci & 1)];
-        uint32_t packed[16];
-        if (live) {
-          float v[32];
-          if constexpr (EPI == EPI_SWIGLU) {
-            float u[32];
-            // FP8: the up half's column scales are read in float4 pieces here
-            // (two preloaded 32-float arrays would not fit in registers)
-            const float4* swb = reinterpret_cast<const float4*>(p.sw + ncol + 128);
-#pragma unroll
-            for (int i4 = 0; i4 < 8; ++i4) {
-              float sb4[4] = {rs, rs, rs, rs};
-              if constexpr (!C::NV) {
-                const float4 w4 = __ldg(swb + i4);
-                sb4[0] = rs * w4.x;
-                sb4[1] = rs * w4.y;
-                sb4[2] = rs * w4.z;
-                sb4[3] = rs * w4.w;
-              }
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int i = 4 * i4 + j;
-                const float sa_ = C::NV ? rs : rs * sw_a[i];
-                v[i] = fmaf(__uint_as_float(ra[i]), sa_, bf16x32_at(bias_a, i));
-                u[i] = fmaf(__uint_as_float(accu[i]), sb4[j], bf16x32_at(bias_b, i));
+            if (normed) {
+              const float4* wp = reinterpret_cast<const float4*>(wgt + 32 * k);
+              const float4* cp =
+                  reinterpret_cast<const float4*>(p.rope_cos + mrow * (QKV_HEAD_DIM / 2) + 16 * k);
+              const float4* snp =
+                  reinterpret_cast<const float4*>(p.rope_sin + mrow * (QKV_HEAD_DIM / 2) + 16 * k);
+  #pragma unroll
+              for (int j4 = 0; j4 < 4; ++j4) {
+                const float4 c4 = __ldg(cp + j4), s4 = __ldg(snp + j4);
+                const float4 w0 = __ldg(wp + 2 * j4), w1 = __ldg(wp + 2 * j4 + 1);
+                const float cs[4] = {c4.x, c4.y, c4.z, c4.w}, sn[4] = {s4.x, s4.y, s4.z, s4.w};
+                const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+  #pragma unroll
+                for (int tt = 0; tt < 4; ++tt) {
+                  const int i = 2 * (4 * j4 + tt);
+                  const float x0 = v[i] * rn * wv[2 * tt], x1 = v[i + 1] * rn * wv[2 * tt + 1];
+                  v[i] = fmaf(x0, cs[tt], -x1 * sn[tt]);
+                  v[i + 1] = fmaf(x0, sn[tt], x1 * cs[tt]);
+                }
               }
             }
-            silu_mul_32(v, u);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              float s_;
-              if constexpr (C::NV)
-                s_ = rs;
-              else
-                s_ = rs * sw_a[i];
-              v[i] = fmaf(__uint_as_float(ra[i]), s_, bf16x32_at(bias_a, i));
-              if constexpr (EPI == EPI_GATED_RES)
-                v[i] = fmaf(bf16x32_at(gate_a, i), v[i], bf16x32_at(res_a, i));
-            }
-            if constexpr (EPI == EPI_BIAS_GELU) {
-              gelu_tanh_32(v);
-            } else if constexpr (EPI == EPI_SPLIT) {
-              if (ncol >= p.split_col) gelu_tanh_32(v);  // uniform per chunk
-            }
-          }
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) packed[i >> 1] = pack_bf16x2(v[i], v[i + 1]);
-        }
-        if constexpr (EPI == EPI_SWIGLU) {
-          // SwiGLU holds two halves per chunk; the next pair is loaded here,
-          // into the same registers
-          if (ci + 1 < nch) {
-            const int cn = chunk_of(ci + 1);
-            tmem_ld_32x32b_x32(tbase + 32 * cn, acc[0]);
-            tmem_ld_32x32b_x32(tbase + 128 + 32 * cn, accu);
-          }
-        }
-        if (!live) continue;
-        if constexpr (OQ) {
-          // two 16-element blocks of the next layer's K: codes for rows < M,
-          // zero scales for the padded rows of the last 128-row block
-          uint2 c0, c1;
-          float a0, a1;
-          const uint32_t sb0 = nvfp4_block(make_uint4(packed[0], packed[1], packed[2], packed[3]),
-                                           make_uint4(packed[4], packed[5], packed[6], packed[7]),
-                                           q_enc, q_G, c0, a0);
-          const uint32_t sb1 =
-              nvfp4_block(make_uint4(packed[8], packed[9], packed[10], packed[11]),
-                          make_uint4(packed[12], packed[13], packed[14], packed[15]), q_enc, q_G,
-                          c1, a1);
-          uint16_t* sfp = reinterpret_cast<uint16_t*>(p.q_sf + sf_offset(m, ocol >> 4, p.q_kchunks));
-          if (row_ok) {
-            *reinterpret_cast<uint4*>(p.q_codes + static_cast<int64_t>(m) * (p.Nout >> 1) +
-                                      (ocol >> 1)) = make_uint4(c0.x, c0.y, c1.x, c1.y);
-            *sfp = static_cast<uint16_t>(sb0 | (sb1 << 8));
-            qmax = fmaxf(qmax, fmaxf(a0, a1));
-          } else if (m < p.q_mpad) {
-            *sfp = 0;
+            uint32_t pk[16];
+  #pragma unroll
+            for (int i = 0; i < 32; i += 2) pk[i >> 1] = pack_bf16x2(v[i], v[i + 1]);
+            store_chunk(pk, h0 + 32 * k);
+          };
+  #pragma unroll 1
+          for (int t = 0; t < nsteps; t += 2) {
+            step(t, ha, hb2);
+            step(t + 1, hb2, ha);
           }
           continue;
         }
-        store_chunk(packed, ocol);
+        // chunk processed at step ci.  SwiGLU with overlapping buffers: the
+        // shared columns are the up half of output chunks 2, 3 in buffer 0 and
+        // the gate half of chunks 0, 1 in buffer 1; every warp holds exactly one
+        // of them and reads it first.
+        auto chunk_of = [&](int ci) {
+          if (MS) return ci;
+          const int k = (C::OVL && buf == 0) ? (nch - 1 - ci) : ci;
+          return half + 2 * k;
+        };
+        constexpr int NCHW = MS ? NCHT : (NCHT + 1) / 2;  // most chunks a warp can have
+        uint32_t acc[2][32];                   // double-buffered accumulator chunk
+        uint32_t accu[32];                     // SwiGLU: the up half
+        tmem_ld_32x32b_x32(tbase + 32 * chunk_of(0), acc[0]);
+        if constexpr (EPI == EPI_SWIGLU) tmem_ld_32x32b_x32(tbase + 128 + 32 * chunk_of(0), accu);
+  #pragma unroll
+        for (int ci = 0; ci < NCHW; ++ci) {
+          if (ci >= nch) break;
+          const int c = chunk_of(ci);
+          const int ncol = nb * BN + 32 * c;  // GEMM column of acc[..][0]
+          const int ocol = (EPI == EPI_SWIGLU) ? nb * (BN / 2) + 32 * c : ncol;  // output column
+          // SwiGLU (N = 256): gate columns ncol.., up columns ncol + 128..
+          const bool live = ncol < p.N;  // past the last column (N % 32 == 0); warp-uniform
+          // per-column and per-row operands: issued before the TMEM wait so the
+          // two latencies overlap
+          uint4 bias_a[4], bias_b[4], gate_a[4], res_a[4];
+          float sw_a[32];
+          if (live) {
+            load_bf16x32_packed(p.bias + ncol, bias_a);
+            if constexpr (!C::NV) load_f32x32(p.sw + ncol, sw_a);
+            if constexpr (EPI == EPI_SWIGLU) {
+              load_bf16x32_packed(p.bias + ncol + 128, bias_b);
+            }
+            if constexpr (EPI == EPI_GATED_RES) {
+              // per-batch gates (CFG-batched tokens): row m uses gate row m / gate_rows
+              const __nv_bfloat16* gp = p.gate + ocol;
+              if (p.gate_rows > 0)
+                gp += static_cast<int64_t>((row_ok ? m : p.M - 1) / p.gate_rows) * p.Nout;
+              load_bf16x32_packed(gp, gate_a);
+              if (row_ok) {
+                load_bf16x32_packed(p.residual + static_cast<int64_t>(m) * p.Nout + ocol, res_a);
+              } else {
+  #pragma unroll
+                for (int i = 0; i < 4; ++i) res_a[i] = make_uint4(0u, 0u, 0u, 0u);
+              }
+            }
+          }
+          tmem_wait_ld();
+          // the next chunk's accumulators stream in while this one is computed
+          if constexpr (EPI != EPI_SWIGLU) {
+            if (ci + 1 < nch) tmem_ld_32x32b_x32(tbase + 32 * chunk_of(ci + 1), acc[(ci + 1) & 1]);
+          }
+          if (C::OVL && ci == 0) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(ovl_l0);
+          }
+          if (ci == nch - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sb->acc_empty[buf]), 0));
+          }
+          const uint32_t* ra = acc[(EPI == EPI_SWIGLU) ? 0 : (ci & 1)];
+          uint32_t packed[16];
+          if (live) {
+            float v[32];
+            if constexpr (EPI == EPI_SWIGLU) {
+              float u[32];
+              // FP8: the up half's column scales are read in float4 pieces here
+              // (two preloaded 32-float arrays would not fit in registers)
+              const float4* swb = reinterpret_cast<const float4*>(p.sw + ncol + 128);
+  #pragma unroll
+              for (int i4 = 0; i4 < 8; ++i4) {
+                float sb4[4] = {rs, rs, rs, rs};
+                if constexpr (!C::NV) {
+                  const float4 w4 = __ldg(swb + i4);
+                  sb4[0] = rs * w4.x;
+                  sb4[1] = rs * w4.y;
+                  sb4[2] = rs * w4.z;
+                  sb4[3] = rs * w4.w;
+                }
+  #pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const int i = 4 * i4 + j;
+                  const float sa_ = C::NV ? rs : rs * sw_a[i];
+                  v[i] = fmaf(__uint_as_float(ra[i]), sa_, bf16x32_at(bias_a, i));
+                  u[i] = fmaf(__uint_as_float(accu[i]), sb4[j], bf16x32_at(bias_b, i));
+                }
+              }
+              silu_mul_32(v, u);
+            } else {
+  #pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                float s_;
+                if constexpr (C::NV)
+                  s_ = rs;
+                else
+                  s_ = rs * sw_a[i];
+                v[i] = fmaf(__uint_as_float(ra[i]), s_, bf16x32_at(bias_a, i));
+                if constexpr (EPI == EPI_GATED_RES)
+                  v[i] = fmaf(bf16x32_at(gate_a, i), v[i], bf16x32_at(res_a, i));
+              }
+              if constexpr (EPI == EPI_BIAS_GELU) {
+                gelu_tanh_32(v);
+              } else if constexpr (EPI == EPI_SPLIT) {
+                if (ncol >= p.split_col) gelu_tanh_32(v);  // uniform per chunk
+              }
+            }
+  #pragma unroll
+            for (int i = 0; i < 32; i += 2) packed[i >> 1] = pack_bf16x2(v[i], v[i + 1]);
+          }
+          if constexpr (EPI == EPI_SWIGLU) {
+            // SwiGLU holds two halves per chunk; the next pair is loaded here,
+            // into the same registers
+            if (ci + 1 < nch) {
+              const int cn = chunk_of(ci + 1);
+              tmem_ld_32x32b_x32(tbase + 32 * cn, acc[0]);
+              tmem_ld_32x32b_x32(tbase + 128 + 32 * cn, accu);
+            }
+          }
+          if (!live) continue;
+          if constexpr (OQ) {
+            // two 16-element blocks of the next layer's K: codes for rows < M,
+            // zero scales for the padded rows of the last 128-row block
+            uint2 c0, c1;
+            float a0, a1;
+            const uint32_t sb0 = nvfp4_block(make_uint4(packed[0], packed[1], packed[2], packed[3]),
+                                             make_uint4(packed[4], packed[5], packed[6], packed[7]),
+                                             q_enc, q_G, c0, a0);
+            const uint32_t sb1 =
+                nvfp4_block(make_uint4(packed[8], packed[9], packed[10], packed[11]),
+                            make_uint4(packed[12], packed[13], packed[14], packed[15]), q_enc, q_G,
+                            c1, a1);
+            uint16_t* sfp = reinterpret_cast<uint16_t*>(p.q_sf + sf_offset(m, ocol >> 4, p.q_kchunks));
+            if (row_ok) {
+              *reinterpret_cast<uint4*>(p.q_codes + static_cast<int64_t>(m) * (p.Nout >> 1) +
+                                        (ocol >> 1)) = make_uint4(c0.x, c0.y, c1.x, c1.y);
+              *sfp = static_cast<uint16_t>(sb0 | (sb1 << 8));
+              qmax = fmaxf(qmax, fmaxf(a0, a1));
+            } else if (m < p.q_mpad) {
+              *sfp = 0;
+            }
+            continue;
+          }
+          store_chunk(packed, ocol);
+        }
       }
     }
     if (lane == 0) bulk_wait_group<0>();
@@ -930,10 +980,19 @@ cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t st) {
 
 int gemm_tile_n(int fmt, int epi) {
   if (fmt == 0) return Cfg<0, 2, EPI_BIAS>::BN;
-  if (fmt == 2) return Cfg<2, 2, EPI_BIAS>::BN;
+  if (fmt == 2) {
+    if (epi == EPI_SWIGLU) return Cfg<2, 2, EPI_SWIGLU>::BN;
+    if (epi == EPI_QKV) return Cfg<2, 2, EPI_QKV>::BN;
+    return Cfg<2, 2, EPI_BIAS>::BN;
+  }
   if (epi == EPI_SWIGLU) return Cfg<1, 2, EPI_SWIGLU>::BN;
   if (epi == EPI_QKV) return Cfg<1, 2, EPI_QKV>::BN;
   return Cfg<1, 2, EPI_BIAS>::BN;
+}
+
+int gemm_tile_msub(int fmt, int epi) {
+  if (fmt == 2 && epi != EPI_SWIGLU && epi != EPI_QKV) return Cfg<2, 2, EPI_BIAS>::MSUB;
+  return 1;
 }
 
 cudaError_t launch_gemm(int fmt, int epi, int cg, int outq, const GemmParams& p, int num_sms,

@@ -265,7 +265,8 @@ ql_status forward_impl(qlinear_t h, const void* codes, const void* scales, int64
   p.Nout = static_cast<int32_t>(h->Nout);
   p.split_col = static_cast<int32_t>(h->d.split_col);
   p.k_blocks = static_cast<int32_t>((kbytes + 127) / 128);
-  p.tiles_m = static_cast<int32_t>((M + 128 * cg - 1) / (128 * cg));
+  const int64_t tile_rows = 128 * cg * gemm_tile_msub(h->d.fmt, h->d.epi);
+  p.tiles_m = static_cast<int32_t>((M + tile_rows - 1) / tile_rows);
   p.tiles_n = static_cast<int32_t>((h->N + h->bn - 1) / h->bn);
   p.group_m = 8;
   p.sf_kchunks_a = static_cast<int32_t>(sf_kchunks(h->K));
