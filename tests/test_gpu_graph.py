@@ -10,7 +10,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("fmt,epi", [("fp8", "bias_gelu"), ("nvfp4", "swiglu"),
-                                     ("nvfp4", "split_bias_gelu")])
+                                     ("nvfp4", "split_bias_gelu"), ("w8a16", "bias")])
 def test_quantize_and_forward_replay_from_a_cuda_graph(fmt, epi):
     import torch
     import precision_gemm_qlinear_b200 as ql

@@ -70,7 +70,7 @@ def test_export_then_import_round_trips(fmt):
 
 
 @pytest.mark.parametrize("variant", [1, 2])
-@pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4", "w8a16"])
 def test_gate_rows_match_oracle_per_group(fmt, variant):
     import torch
     import precision_gemm_qlinear_b200 as ql

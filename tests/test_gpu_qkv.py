@@ -43,7 +43,7 @@ def _run(fmt, M, N, K, seed, variant, eps=1e-6):
 
 
 @pytest.mark.parametrize("variant", [1, 2])
-@pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4", "w8a16"])
 def test_qkv_norm_rope_matches_oracle(fmt, variant):
     # 3 ragged M tiles (one CTA) / 2 pair tiles; q, k, v of two heads each
     got, ref = _run(fmt, 300, 768, 256, 21, variant)
@@ -52,7 +52,7 @@ def test_qkv_norm_rope_matches_oracle(fmt, variant):
     assert np.all(np.abs(np.sqrt(np.mean(ref[:, :512] ** 2, axis=1)) - 1.0) < 0.5)
 
 
-@pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4", "w8a16"])
 def test_qkv_norm_rope_more_heads_and_tiles(fmt):
     got, ref = _run(fmt, 520, 1536, 512, 22, 0, eps=1e-3)
     assert_close(got, ref)
