@@ -84,14 +84,14 @@ struct Cfg {
   static constexpr int EPI_PASSES = 8 / EPI_WARPS;
   static constexpr int CONV_WARPS = W16 ? 4 : 0;
   static constexpr int THREADS = 64 + 32 * (EPI_WARPS + CONV_WARPS);
-  // Tile N: 256, except NVFP4 without SwiGLU, where 224 lets two fp32
-  // accumulators (2 x 224 TMEM columns) and the 48 scale-factor columns fit
-  // in the 512 columns side by side.
+  // Tile N: 256 (NVFP4 included: its eight scale-factor copies per stage
+  // cost the same whatever N, so the widest MMA amortizes them best; the
+  // two accumulators then overlap in TMEM, see below).
   // FMT 2 with an epilogue that does not need 256-column tiles: each CTA
   // computes MSUB = 2 row subtiles against the same converted weight stage
   // (tile (2 x 128 CG) x 128), halving the conversion per MMA.
   static constexpr int MSUB = (FMT == 2 && EPI != EPI_SWIGLU && EPI != EPI_QKV) ? 2 : 1;
-  static constexpr int BN = (NV && EPI != EPI_SWIGLU && EPI != EPI_QKV) ? 224 : (MSUB == 2 ? 128 : 256);
+  static constexpr int BN = MSUB == 2 ? 128 : 256;
   static constexpr int A_BYTES = MSUB * A_TILE_BYTES;  // this stage's rows of A
   static constexpr int B_BYTES = (BN / CG) * BK_BYTES;  // this CTA's rows of B
   static constexpr int SFA_BYTES = NV ? 2048 : 0;       // 4 atoms (one per MMA K step)
@@ -108,10 +108,10 @@ struct Cfg {
   static constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;  // + barriers + alignment slack
   // TMEM columns: FP8 -> two disjoint 256-column accumulators.  NVFP4 ->
   // the scale factors of the current stage live in [448, 496) (A in 4 x 4
-  // columns, B in 4 x 8, one group per 64-element MMA step); with N = 224 the
-  // accumulators are [0,224) and [224,448); with N = 256 (SwiGLU) they are
-  // [0,256) and [192,448), overlapping in [192,256), and the epilogue reads
-  // the shared columns first and releases them early.
+  // columns, B in 4 x 8, one group per 64-element MMA step) and the two
+  // 256-column accumulators are [0,256) and [192,448), overlapping in
+  // [192,256); the epilogue reads the shared columns first and releases them
+  // early.
   static constexpr bool OVL = NV && BN == 256;
   static constexpr uint32_t ACC1 = OVL ? 192 : MSUB * BN;
   static constexpr uint32_t SFA_COL = 448;

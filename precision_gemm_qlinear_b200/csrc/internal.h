@@ -40,7 +40,7 @@ __host__ __device__ __forceinline__ int64_t sf_bytes(int64_t rows, int64_t K) {
 
 // Scale-factor layout of the weight (B) operand, fed to TMEM by one
 // tcgen05.cp.128x256b per 64-element MMA step: for every N tile of `bn` rows
-// (256, or 224), every stage of 256 K-elements and every MMA step j (0..3)
+// (the GEMM tile N, 256), every stage of 256 K-elements and every MMA step j (0..3)
 // there is a 4096-byte chunk of 128 rows x 32 bytes.  Row (TMEM lane)
 // l = 32 q + r0 holds, in word w (0..7), the 4 scales of weight row
 // bn * tile + 32 w + r0 for that step -- the same for every q (the
@@ -48,7 +48,8 @@ __host__ __device__ __forceinline__ int64_t sf_bytes(int64_t rows, int64_t K) {
 // Chunks are ordered [tile][stage][j]; the 32-byte rows are stored in the
 // unswizzled K-major core-matrix order the copy expects: 8-row groups 256
 // bytes apart, the two 16-byte halves of a row 128 bytes apart, rows of a
-// group 16 bytes apart.  Words past the tile (bn = 224: word 7) are zero.
+// group 16 bytes apart.  Words of rows past N (and of rows past bn, for a
+// tile narrower than 256) are zero.
 __host__ __device__ __forceinline__ int64_t sfb_stages(int64_t K) { return (K + 255) / 256; }
 __host__ __device__ __forceinline__ int64_t sfb_bytes(int64_t rows, int64_t K, int64_t bn) {
   return ((rows + bn - 1) / bn) * sfb_stages(K) * 4 * 4096;

@@ -40,7 +40,7 @@ struct qlinear_s {
   float qk_eps;        // QKV epilogue: RMS normalization epsilon
   RowMap map;
   int32_t fault_mode;  // test hook, see qlinear_debug_set_fault
-  int32_t bn;          // N of the GEMM tile (256, or 224 for NVFP4 without SwiGLU)
+  int32_t bn;          // N of the GEMM tile (256, or 128 for weight-only bias-type layers)
   CUtensorMap tmB1;    // weight codes, box 128 B x 256 rows (one CTA per tile)
   CUtensorMap tmB2;    // weight codes, box 128 B x 128 rows (CTA pair per tile)
   CUtensorMap tmSFB;   // NVFP4: weight SF atoms as 2048-byte rows (CTA pair)
@@ -422,7 +422,7 @@ ql_status qlinear_create(const ql_desc* desc, const void* w_bf16, const void* bi
     e = launch_quant_fp8_rows(w_bf16, h->N, h->K, h->K, h->wcodes, h->wscale, h->map, h->num_sms,
                               st);
   } else if (e == cudaSuccess) {
-    // unused scale words (rows past N, word 7 of a 224-row tile) stay zero
+    // unused scale words (rows past N) stay zero
     e = cudaMemsetAsync(h->wsf, 0, sfb_bytes(h->N, h->K, h->bn) + 16, st);
     if (e == cudaSuccess) e = launch_tensor_amax(w_bf16, h->N * h->K, h->wamax, h->num_sms, st);
     if (e == cudaSuccess)

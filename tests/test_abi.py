@@ -39,7 +39,7 @@ def test_status_strings_and_version():
     ("fp8", "bias", 9200, 3072, False),      # N % 32
     ("nvfp4", "bias", 9216, 3072, True),
     ("nvfp4", "bias", 9216, 3056, False),    # K % 32
-    ("nvfp4", "bias", 9248, 3072, True),     # N % 32 (224-column tiles)
+    ("nvfp4", "bias", 9248, 3072, True),     # N % 32 (ragged last tile)
     ("nvfp4", "swiglu", 9248, 3072, False),  # SwiGLU needs N % 256
     ("fp8", "swiglu", 16384, 3072, True),
     ("fp8", "swiglu", 16416, 3072, False),   # SwiGLU needs N % 256

@@ -39,7 +39,8 @@ def test_weight_sf_layout_words_tile_the_buffer(N, K):
 
 @pytest.mark.parametrize("N,K", [(224, 256), (768, 3072), (21504, 512)])
 def test_weight_sf_layout_224_row_tiles(N, K):
-    # 224-row tiles use words 0..6 of every row: the slots are distinct and
+    # the layout also serves tiles narrower than 256 rows: 224-row tiles use
+    # words 0..6 of every row, the slots are distinct and
     # the unused word 7 of each row is exactly what is left over
     off = sfb_word_offsets(N, K, 224).ravel()
     tiles = (N + 223) // 224
