@@ -20,6 +20,7 @@ the host cores, on a bounded row sample per step.
 """
 import argparse
 import hashlib
+import re
 import json
 import os
 import sys
@@ -78,11 +79,21 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def gemm_source_sha():
+def strip_comments(src):
+    """C/C++ source without comments, trailing blanks or blank lines, so that
+    the fingerprint below changes with the code only (the kernel sources hold
+    no comment markers inside string literals)."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(ln.rstrip() for ln in src.splitlines() if ln.strip())
+
+
+def gemm_source_sha(root=None):
+    """Fingerprint of the GEMM kernel's code (comments excluded)."""
     h = hashlib.sha256()
     for p in GEMM_SOURCES:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(root or ROOT, p)) as f:
+            h.update(strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -8,18 +8,23 @@
 //          mbarrier, and the leader's single MMA thread drives both tensor
 //          cores.  Per SM, 32 KB of operands feed 512 cycles of FP8 MMA.
 //   CG = 1: one CTA computes a 128 x 256 tile (used when M <= 128).
+//   Weight-only layers with bias-type epilogues compute two such row
+//   subtiles per CTA against 128-column weight tiles (512 x 128 per pair).
 // Roles (10 warps):
 //   warp 0      TMA producer: A / B tiles (128-byte swizzle) and, for NVFP4,
 //               the block-scale atoms, into an S-stage shared-memory ring
 //               guarded by full/empty mbarriers;
 //   warp 1      TMEM allocation (512 columns) and, in the leader CTA, the MMA
 //               issuer (kind::f8f6f4 for FP8; kind::mxf4nvf4 with block16 E4M3
-//               scales for NVFP4, scales staged to TMEM with tcgen05.cp) into a
-//               double-buffered fp32 TMEM accumulator;
+//               scales for NVFP4, scales staged to TMEM with tcgen05.cp;
+//               kind::f16 for weight-only layers) into a double-buffered fp32
+//               TMEM accumulator;
 //   warps 2..9  epilogue: tcgen05.ld -> registers -> dequant scale, bias,
 //               activation / gated residual -> bf16 -> swizzled shared staging
 //               -> TMA store.  Two warps share each TMEM sub-partition (32
-//               rows) and split its 256 columns.
+//               rows) and split its columns.
+//   Weight-only layers: warps 2..5 are the epilogue (one per sub-partition,
+//   two passes) and warps 6..9 expand the FP8 weight stages to bf16.
 // Tiles are visited in groups of `group_m` M-tiles for L2 reuse.  Every
 // mbarrier wait is bounded (one second of %globaltimer); on expiry the CTA
 // records an error code, drains what it issued and exits cleanly (no trap).

@@ -27,3 +27,13 @@ def test_cpu_baseline_runs_for_every_format_and_epilogue():
         wl = bench.with_tokens(WORKLOADS[name], 8)
         tflops, rows, dt, cores = bench.cpu_baseline(wl, 0.01)
         assert tflops > 0 and 1 <= rows <= 8 and cores >= 1
+
+
+def test_kernel_fingerprint_follows_code_not_comments():
+    # the recorded DRAM traffic is reported only while the kernel's code is
+    # the one that was profiled: comment edits keep the fingerprint, code
+    # edits change it
+    src = "int a; // note\n/* block\n comment */ int b;\n\n"
+    assert bench.strip_comments(src) == bench.strip_comments("int a;   \n int b; // other\n")
+    assert bench.strip_comments(src) != bench.strip_comments("int a; int c;\n")
+    assert len(bench.gemm_source_sha()) == 16
