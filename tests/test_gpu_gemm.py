@@ -91,3 +91,66 @@ def test_many_tiles_per_cta(fmt, variant):
     got, ref = _run(fmt, "split_bias_gelu", M, N, K, x_kind="t", rows=rows, split_col=1024,
                     variant=variant)
     assert_close(got, ref, f"many tiles {fmt} v{variant}")
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4", "w8a16"])
+def test_zero_activation_rows_give_the_bias(fmt):
+    # an all-zero token has amax 0: its scale (FP8) or block scales (NVFP4)
+    # are 0, its codes are 0 and its output row is exactly the bias; the
+    # other rows are unaffected (whole output against the oracle)
+    import torch
+    import precision_gemm_qlinear_b200 as ql
+    M, N, K = 300, 512, 512
+    x = draw("normal", (M, K), 51, "x")
+    zero_rows = [0, 5, 130, 255, 256, M - 1]
+    x[zero_rows] = 0
+    w = draw("normal", (N, K), 51, "w", std=0.02)
+    b = draw("normal", (N,), 51, "bias", std=0.01)
+    lay = ql.QLinear(fmt, "bias", to_dev_bf16(w), to_dev_bf16(b))
+    out = lay(to_dev_bf16(x))
+    torch.cuda.synchronize()
+    assert lay.check() == 0
+    bits = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    for r in zero_rows:
+        assert np.array_equal(bits[r], b), f"row {r}"
+    ref = oracle.qlinear_reference(fmt, "bias", x, w, bias=b)["out"]
+    assert_close(from_dev_bf16(out), ref, f"zero rows {fmt}")
+
+
+def test_nvfp4_all_zero_tensor():
+    # tensor amax 0: the global scale and every block scale are 0, every code
+    # is 0, and the output is the bias broadcast over the tokens
+    import torch
+    import precision_gemm_qlinear_b200 as ql
+    M, N, K = 200, 256, 256
+    w = draw("normal", (N, K), 52, "w", std=0.02)
+    b = draw("normal", (N,), 52, "bias", std=0.01)
+    lay = ql.QLinear("nvfp4", "bias_gelu", to_dev_bf16(w), to_dev_bf16(b))
+    x = np.zeros((M, K), np.uint16)
+    out = lay(to_dev_bf16(x))
+    torch.cuda.synchronize()
+    assert lay.check() == 0
+    ref = oracle.qlinear_reference("nvfp4", "bias_gelu", x, w, bias=b)["out"]
+    assert_close(from_dev_bf16(out), ref, "all-zero NVFP4")
+    bits = out.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.all(bits == bits[0])  # every token the same row: gelu(bias)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4", "w8a16"])
+def test_empty_batch_is_a_no_op(fmt):
+    # M = 0: quantize and forward return success and write nothing
+    import torch
+    import precision_gemm_qlinear_b200 as ql
+    N, K = 256, 256
+    lay = ql.QLinear(fmt, "bias_gelu", to_dev_bf16(draw("normal", (N, K), 53, "w", std=0.02)))
+    x = to_dev_bf16(draw("normal", (4, K), 53, "x"))
+    codes, scales = lay.act_buffers(4)
+    codes.fill_(0xA5)
+    scales.fill_(0xA5)
+    out = torch.full((4, N), 7.0, dtype=torch.bfloat16, device="cuda")
+    lay.quantize(x[:0], codes, scales)
+    lay.forward_codes(x if fmt == "w8a16" else codes, scales, 0, out)
+    torch.cuda.synchronize()
+    assert lay.check() == 0
+    assert bool((codes == 0xA5).all()) and bool((scales == 0xA5).all())
+    assert bool((out == 7.0).all())
