@@ -153,13 +153,17 @@ __device__ __forceinline__ void tile_coords(int t, const GemmParams& p, int& mb,
 // Bounded wait on an mbarrier phase.  Returns false when the CTA is aborting
 // (another role gave up) or this wait exceeded the limit (then it raises the
 // abort flag and records `code` in the device error word).
+template <bool CLUSTER_ACQ = false>
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, SmemBars* sb,
                                          uint32_t* err, uint32_t code) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
+  auto try_wait = [&]() {
+    return CLUSTER_ACQ ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity);
+  };
+  if (try_wait()) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(a, parity)) return true;
+    if (try_wait()) return true;
     if ((it & 31) == 0) {
       if (sb->abort_flag) return false;
       if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
@@ -454,7 +458,7 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
           }
           if constexpr (C::W16) {
             // both CTAs' converter warps have written this stage's bf16 B
-            if (!wait_bar(&sb->conv_done[stage], phase, sb, p.err, ERR_WAIT_MMA)) {
+            if (!wait_bar<true>(&sb->conv_done[stage], phase, sb, p.err, ERR_WAIT_MMA)) {
               ok = false;
               break;
             }
@@ -598,7 +602,7 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
           }
           fence_proxy_async_smem();  // generic-proxy writes -> the tensor core's reads
           __syncwarp();
-          if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(done_l0 + 8u * stage);
+          if ((threadIdx.x & 31) == 0) mbar_arrive_cluster_smem_release(done_l0 + 8u * stage);
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1;

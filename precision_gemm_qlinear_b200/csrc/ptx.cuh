@@ -268,6 +268,33 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
                : "memory");
 }
 
+// Publish this thread's writes to its own CTA's shared memory to a thread of
+// the cluster that waits on the mbarrier at `cluster_addr` (possibly in the
+// peer CTA) with a cluster-scope acquire: a release fence restricted to
+// shared::cta operations, then a relaxed arrive.  The restricted fence only
+// has to order shared-memory stores, which makes it far cheaper than the
+// arrive's own release semantics (those order every prior memory operation).
+__device__ __forceinline__ void mbar_arrive_cluster_smem_release(uint32_t cluster_addr) {
+  asm volatile(
+      "fence.release.sync_restrict::shared::cta.cluster;\n\t"
+      "mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+      : "memory");
+}
+
+// Parity wait with cluster-scope acquire (the arrivals come from either CTA
+// of the pair).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // 2-D tiled load into this CTA's shared memory whose completion is counted on
 // the mbarrier of the pair's leader CTA (`bar` is a shared::cluster address).
 // No multicast: every CTA of the pair loads its own half.
