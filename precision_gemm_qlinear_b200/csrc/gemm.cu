@@ -8,8 +8,8 @@
 //          mbarrier, and the leader's single MMA thread drives both tensor
 //          cores.  Per SM, 32 KB of operands feed 512 cycles of FP8 MMA.
 //   CG = 1: one CTA computes a 128 x 256 tile (used when M <= 128).
-//   Weight-only layers with bias-type epilogues compute two such row
-//   subtiles per CTA against 128-column weight tiles (512 x 128 per pair).
+//   The kernel can also compute two row subtiles per CTA against one
+//   128-column weight tile (Cfg::MSUB); the current configuration uses one.
 // Roles (10 warps):
 //   warp 0      TMA producer: A / B tiles (128-byte swizzle) and, for NVFP4,
 //               the block-scale atoms, into an S-stage shared-memory ring
@@ -92,10 +92,13 @@ struct Cfg {
   // Tile N: 256 (NVFP4 included: its eight scale-factor copies per stage
   // cost the same whatever N, so the widest MMA amortizes them best; the
   // two accumulators then overlap in TMEM, see below).
-  // FMT 2 with an epilogue that does not need 256-column tiles: each CTA
-  // computes MSUB = 2 row subtiles against the same converted weight stage
-  // (tile (2 x 128 CG) x 128), halving the conversion per MMA.
-  static constexpr int MSUB = (FMT == 2 && EPI != EPI_SWIGLU && EPI != EPI_QKV) ? 2 : 1;
+  // MSUB row subtiles per CTA against one converted weight stage (tile
+  // (MSUB x 128 CG) x 128 for MSUB = 2, halving the conversion per MMA).
+  // The kernel supports 2 for weight-only layers whose epilogue does not
+  // need 256-column tiles, but one subtile with a fifth operand stage (which
+  // two subtiles leave no room for) is faster since the converted stages
+  // are published cheaply, so 1 is used throughout.
+  static constexpr int MSUB = 1;
   static constexpr int BN = MSUB == 2 ? 128 : 256;
   static constexpr int A_BYTES = MSUB * A_TILE_BYTES;  // this stage's rows of A
   static constexpr int B_BYTES = (BN / CG) * BK_BYTES;  // this CTA's rows of B
@@ -103,7 +106,7 @@ struct Cfg {
   static constexpr int SFB_BYTES = NV ? 16384 : 0;      // 4 replicated 4 KB chunks (all 256 B rows)
   static constexpr int B8_BYTES = W16 ? (BN / CG) * 64 : 0;  // raw FP8 weights, 64 per row
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES + B8_BYTES;
-  static constexpr int STAGES = NV ? (PAIR ? 4 : 3) : (W16 ? (PAIR ? 4 : 3) : (PAIR ? 6 : 4));
+  static constexpr int STAGES = NV ? (PAIR ? 4 : 3) : (W16 ? (PAIR ? 5 : 3) : (PAIR ? 6 : 4));
   // staging buffers per epilogue warp: two unless that breaks the budget
   static constexpr int NBUF =
       (STAGES * STAGE_BYTES + EPI_WARPS * 2 * STAGING_BYTES + 512 + 1024 <= 232448) ? 2 : 1;

@@ -162,8 +162,9 @@ cudaError_t launch_gemm(int fmt, int epi, int cg, int outq, const GemmParams& p,
                         cudaStream_t st);
 // N of the GEMM tile for a format / epilogue (the weight scale layout uses it).
 int gemm_tile_n(int fmt, int epi);
-// Row subtiles per CTA (2 for weight-only layers with 128-column tiles): a
-// tile covers 128 * cg * msub rows.
+// Row subtiles per CTA (the kernel supports 2 for weight-only layers with
+// 128-column tiles; every configuration in use has 1): a tile covers
+// 128 * cg * msub rows.
 int gemm_tile_msub(int fmt, int epi);
 
 // Error codes written to the device error word by the GEMM watchdog.

@@ -50,13 +50,12 @@ def test_w8a16_ragged_shapes():
 
 @pytest.mark.parametrize("epi", ["bias", "bias_gated_residual"])
 @pytest.mark.parametrize("variant", [1, 2])
-def test_w8a16_many_tiles_with_an_empty_row_subtile(epi, variant):
-    # bias-type layers compute two row subtiles per tile (512 rows per CTA
-    # pair, 256 per single CTA) against 128-column weight tiles: M = 1100
-    # leaves the last tile's second subtile without rows (pairs) or partly
-    # filled (single CTAs); N = 544 ends in a 32-column ragged tile; K = 1088
-    # is 17 stages, so the 4- (3-) stage ring wraps several times and every
-    # converter warp converts stages of several tiles
+def test_w8a16_many_tiles_ragged_in_m_n_and_k(epi, variant):
+    # M = 1100 ends in a partly filled row tile; N = 544 ends in a 32-column
+    # ragged tile; K = 1088 is 17 stages, so the 5- (pairs) or 3-stage
+    # (single CTAs) ring wraps several times, the converter warp that owns two
+    # of the five stages alternates between them, and every converter warp
+    # converts stages of several tiles
     got, ref = _run(epi, 1100, 544, 1088, 44, variant)
     assert_close(got, ref)
 
