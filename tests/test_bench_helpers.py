@@ -37,3 +37,42 @@ def test_kernel_fingerprint_follows_code_not_comments():
     assert bench.strip_comments(src) == bench.strip_comments("int a;   \n int b; // other\n")
     assert bench.strip_comments(src) != bench.strip_comments("int a; int c;\n")
     assert len(bench.gemm_source_sha()) == 16
+
+
+def _bench(args, env_extra=None):
+    import json
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), *args], env=env,
+                       capture_output=True, text=True, timeout=300, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    return [json.loads(ln) for ln in lines]
+
+
+def test_reference_arm_prints_the_contract_line():
+    # the reference arm is the oracle timed on the host cores, on the same
+    # metric and workload as the GPU arm
+    (line,) = _bench(["--impl", "reference", "--steps", "2", "--warmup", "1",
+                      "--workload", "tiny_fp8"])
+    assert line["impl"] == "reference"
+    assert line["metric"] == "quantized DiT linear TFLOP/s at FLUX shapes"
+    assert line["unit"] == "TFLOP/s" and line["higher_is_better"] is True
+    assert line["steps"] == 2 and line["warmup"] == 1 and line["value"] > 0
+    assert line["config"]["workload"] == "tiny_fp8"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    # under a multi-rank launch the other ranks exit cleanly without work
+    assert _bench(["--impl", "reference", "--steps", "1", "--warmup", "0",
+                   "--workload", "tiny_fp8"],
+                  {"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"}) == []
