@@ -31,6 +31,21 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
+def _need(t, name, dtype, shape=None):
+    """Refuse, before any launch, a tensor the kernels cannot read: not on
+    the GPU, of another dtype, not contiguous, or of the wrong shape."""
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (got device {t.device})")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype} (got {t.dtype})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+
+
 class QLinear:
     """One quantized linear layer: weights quantized once, activations per call.
 
@@ -40,8 +55,11 @@ class QLinear:
 
     def __init__(self, fmt, epi, w, bias=None, split_col=0, variant=0, stream=None):
         import torch
-        assert w.is_cuda and w.dtype == torch.bfloat16 and w.is_contiguous()
+        _need(w, "w", torch.bfloat16)
+        if w.dim() != 2:
+            raise ValueError(f"w must be 2-D [N, K] (got {tuple(w.shape)})")
         N, K = w.shape
+        _need(bias, "bias", torch.bfloat16, (N,))
         self.fmt, self.epi, self.N, self.K = fmt, epi, int(N), int(K)
         self.desc = make_desc(fmt, epi, N, K, split_col, variant)
         nbytes = qlinear_weight_bytes(self.desc)
@@ -57,8 +75,11 @@ class QLinear:
         returns: codes uint8 CUDA [N, K] (FP8) or [N, K/2] (NVFP4); scales
         fp32 [N] (FP8) or uint8 [N, K/16] E4M3 block scales (NVFP4); G."""
         import torch
+        _need(codes, "codes", torch.uint8)
+        _need(scales, "scales", torch.float32 if fmt != "nvfp4" else torch.uint8)
         self = cls.__new__(cls)
         N = int(codes.shape[0])
+        _need(bias, "bias", torch.bfloat16, (N,))
         K = int(codes.shape[1]) * (2 if fmt == "nvfp4" else 1)
         self.fmt, self.epi, self.N, self.K = fmt, epi, N, K
         self.desc = make_desc(fmt, epi, N, K, split_col, variant)
@@ -113,7 +134,13 @@ class QLinear:
 
     def __call__(self, x, residual=None, gate=None, out=None, bufs=None, stream=None):
         import torch
+        _need(x, "x", torch.bfloat16)
+        if x.dim() != 2 or x.shape[1] != self.K:
+            raise ValueError(f"x must be [M, {self.K}] (got {tuple(x.shape)})")
         M = x.shape[0]
+        _need(residual, "residual", torch.bfloat16, (M, self.Nout))
+        _need(gate, "gate", torch.bfloat16, (self.Nout,))
+        _need(out, "out", torch.bfloat16, (M, self.Nout))
         codes, scales = bufs if bufs is not None else self.act_buffers(M, x.device)
         if out is None:
             out = torch.empty((M, self.Nout), dtype=torch.bfloat16, device=x.device)

@@ -102,3 +102,34 @@ def test_null_handle_calls():
     assert L.qlinear_destroy(None) == _abi.QL_ERR_INVALID_ARG
     c, s = ctypes.c_size_t(), ctypes.c_size_t()
     assert L.qlinear_act_bytes(None, 4, ctypes.byref(c), ctypes.byref(s)) == _abi.QL_ERR_INVALID_ARG
+
+
+def test_binding_refuses_tensors_the_kernels_cannot_read():
+    # checked in Python before any CUDA call: a host tensor, a wrong dtype or
+    # a wrong shape never reaches a kernel as a pointer
+    import pytest
+    import torch
+    import precision_gemm_qlinear_b200 as ql
+    from precision_gemm_qlinear_b200 import _need
+    with pytest.raises(TypeError, match="CUDA"):
+        ql.QLinear("fp8", "bias", torch.zeros(256, 256, dtype=torch.bfloat16))
+    with pytest.raises(TypeError, match="CUDA"):
+        ql.QLinear.from_quantized("fp8", "bias", torch.zeros(256, 256, dtype=torch.uint8),
+                                  torch.ones(256))
+
+    class FakeCuda:  # the checks only look at these attributes
+        def __init__(self, dtype, shape, contiguous=True):
+            self.is_cuda, self.dtype, self.shape = True, dtype, shape
+            self._c = contiguous
+            self.device = "cuda:0"
+
+        def is_contiguous(self):
+            return self._c
+
+    _need(FakeCuda(torch.bfloat16, (8, 4)), "x", torch.bfloat16, (8, 4))
+    with pytest.raises(TypeError, match="float32"):
+        _need(FakeCuda(torch.float32, (8, 4)), "x", torch.bfloat16)
+    with pytest.raises(ValueError, match="contiguous"):
+        _need(FakeCuda(torch.bfloat16, (8, 4), contiguous=False), "x", torch.bfloat16)
+    with pytest.raises(ValueError, match="shape"):
+        _need(FakeCuda(torch.bfloat16, (8, 5)), "gate", torch.bfloat16, (8, 4))
