@@ -35,6 +35,8 @@
 // matmul runs on the 8-bit tensor cores).  wavespeed.ai "Arquitectura de GPU
 // Blackwell de NVIDIA: B200" names the features used here: TMEM, CTA pairs
 // that share tensor-core work, 5th-generation tensor cores with FP8/FP4.
+#include <atomic>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -959,13 +961,18 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
 template <int FMT, int EPI, int CG, int OQ>
 cudaError_t launch_one(const GemmParams& p, int num_sms, cudaStream_t st) {
   using C = Cfg<FMT, CG, EPI>;
-  static bool attr_set = false;
+  // the shared-memory opt-in is a per-device function attribute: set it once
+  // for each device this process launches on (devices past 63 every time)
+  static std::atomic<uint64_t> attr_devices{0};
   auto kern = qgemm_kernel<FMT, EPI, CG, OQ>;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
+  if (!(attr_devices.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_devices.fetch_or(bit, std::memory_order_release);
   }
   const int tiles = p.tiles_m * p.tiles_n;
   const int units = num_sms / CG;
