@@ -549,9 +549,10 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
   } else if (warp >= 2 + C::EPI_WARPS) {
     // ------------------------ FMT 2: FP8 weight stage -> bf16 MMA operand
     // Four warps per CTA, each owning the stages s with s % 4 == its index
-    // (with three stages the fourth warp has none): a warp converts a whole
-    // stage, so the fence that publishes one stage to the tensor core
-    // overlaps the other warps' conversion of the next ones.  Owning whole
+    // (with five stages warp 0 owns two, with three warp 3 has none): a warp
+    // converts a whole stage, so the publication of one stage to the tensor
+    // core (proxy fence, release, arrive) overlaps the other warps'
+    // conversion of the next ones.  Owning whole
     // stages keeps every warp's waits on a stage's barrier in the order of
     // its phases (a parity wait must never run two phases ahead).  Each lane takes
     // 16-byte chunks (16 E4M3 codes) of the raw stage -- consecutive lanes
