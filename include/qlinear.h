@@ -278,6 +278,24 @@ QL_API ql_status qlinear_destroy(qlinear_t h);
  * Host only, no CUDA call. */
 QL_API ql_status qlinear_debug_set_fault(qlinear_t h, int32_t mode);
 
+/* Test hook for the device encoders (no counterpart on the pages): runs the
+ * conversions that the quantize kernels and the NVFP4-output epilogue use on
+ * caller-chosen values, so that tests can compare every code with a
+ * reference encoder (ties, saturation, subnormals, non-finite inputs).
+ *   mode 0: in = device fp32 [n] -> out = device u8 [n], E4M3 codes (round to
+ *           nearest even, saturating to +-448; NaN stays NaN);
+ *   mode 1: in = device fp32 [n] -> out = device u8 [n], one E2M1 code per
+ *           byte (low nibble; saturating to +-6);
+ *   mode 2: in = device bf16 [n], n % 16 == 0, 16-element blocks quantized
+ *           to NVFP4 against the tensor amax in the device fp32 scalar
+ *           `amax` (G = amax/2688, block scale E4M3(amax_b * 448/amax));
+ *           out = device u8 [n/2 + n/16]: the codes of every block (8 bytes
+ *           each, element 2j in the low nibble), then one block-scale byte
+ *           per block.
+ *   in and out 16-byte aligned.  Enqueued on `stream`, no host sync. */
+QL_API ql_status qlinear_debug_encode(int32_t mode, const void* in, int64_t n, const float* amax,
+                                      void* out, void* stream);
+
 /* Static description of a status code. */
 QL_API const char* qlinear_status_string(ql_status s);
 

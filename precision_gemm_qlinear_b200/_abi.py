@@ -21,7 +21,8 @@ EXPORTS = ("qlinear_weight_bytes", "qlinear_create", "qlinear_create_prequantize
            "qlinear_act_bytes", "qlinear_out_features",
            "qlinear_quantize_act", "qlinear_quantize_act_noalloc", "qlinear_forward",
            "qlinear_forward_gate_rows", "qlinear_forward_nvfp4_out", "qlinear_forward_rope",
-           "qlinear_set_qk_norm", "qlinear_export_weights", "qlinear_check", "qlinear_debug_set_fault", "qlinear_destroy",
+           "qlinear_set_qk_norm", "qlinear_export_weights", "qlinear_check", "qlinear_debug_set_fault",
+           "qlinear_debug_encode", "qlinear_destroy",
            "qlinear_status_string", "qlinear_abi_version")
 
 
@@ -68,6 +69,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.qlinear_export_weights.argtypes = [P, P, P, ctypes.POINTER(ctypes.c_float), P]
     L.qlinear_check.argtypes = [P, P]
     L.qlinear_debug_set_fault.argtypes = [P, ctypes.c_int32]
+    L.qlinear_debug_encode.argtypes = [ctypes.c_int32, P, i64, P, P, P]
     L.qlinear_destroy.argtypes = [P]
     L.qlinear_status_string.argtypes = [st]
     L.qlinear_status_string.restype = ctypes.c_char_p
@@ -221,3 +223,12 @@ def qlinear_destroy(h):
 
 def qlinear_debug_set_fault(h, mode):
     _ck("qlinear_debug_set_fault", load().qlinear_debug_set_fault(h, mode))
+
+
+def qlinear_debug_encode(mode, in_ptr, n, amax_ptr, out_ptr, stream=0, check=True):
+    """Device encoders on given values (test hook): mode 0 E4M3, 1 E2M1 of
+    fp32 in[n]; mode 2 NVFP4 blocks of bf16 in[n] against the amax scalar."""
+    s = load().qlinear_debug_encode(int(mode), in_ptr, int(n), amax_ptr, out_ptr, stream)
+    if check:
+        _ck("qlinear_debug_encode", s)
+    return s

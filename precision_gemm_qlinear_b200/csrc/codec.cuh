@@ -40,6 +40,14 @@ __device__ __forceinline__ uint32_t e2m1_4(const uint2& w, float inv) {
   return b0 | (b1 << 8);
 }
 
+// NVFP4 tensor factors from the tensor amax A: the global (decode) scale
+// G = A/2688 (2688 = 448 * 6, the largest E4M3 block scale times the largest
+// E2M1 value) and the block-scale encode factor enc = 448/A (0 when A is 0).
+__device__ __forceinline__ void nvfp4_tensor_factors(float A, float& G, float& enc) {
+  G = __fdiv_rn(A, 2688.f);
+  enc = A > 0.f ? __fdiv_rn(448.f, A) : 0.f;
+}
+
 // NVFP4 block of 16 elements (v0: elements 0-7, v1: 8-15) against the tensor
 // factors G = A/2688 and enc = 448/A: E4M3 block scale sb = E4M3(amax_b * enc),
 // element factor inv = 1/(dec(sb) * G) (0 when that is 0), 8 bytes of codes;

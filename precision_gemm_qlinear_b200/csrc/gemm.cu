@@ -631,9 +631,7 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
     // |value| this thread quantizes (for the observed amax)
     float q_G = 0.f, q_enc = 0.f, qmax = 0.f;
     if constexpr (OQ) {
-      const float qA = __ldg(p.q_amax);
-      q_G = __fdiv_rn(qA, 2688.f);
-      q_enc = qA > 0.f ? __fdiv_rn(448.f, qA) : 0.f;
+      nvfp4_tensor_factors(__ldg(p.q_amax), q_G, q_enc);
       if (blockIdx.x == 0 && ew == 0 && lane == 0) *p.q_g = q_G;
     }
     for (int t = unit; t < num_tiles; t += nunits, ++local) {

@@ -101,6 +101,11 @@ cudaError_t launch_tensor_amax(const void* x, int64_t n_elems, uint32_t* amax_bi
 cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
                                uint8_t* sf, int sf_layout, int64_t bn, const uint32_t* amax_bits,
                                float* g_out, RowMap map, cudaStream_t st);
+// Test hook: mode 0 / 1 E4M3 / E2M1 codes of fp32 in[n]; mode 2 NVFP4 blocks
+// of bf16 in[n] (n % 16 == 0) against the tensor amax *amax (codes, then
+// the block scales).
+cudaError_t launch_debug_encode(int mode, const void* in, int64_t n, const float* amax,
+                                uint8_t* out, cudaStream_t st);
 cudaError_t launch_permute_bias(const void* src, void* dst, int64_t N, RowMap map,
                                 cudaStream_t st);
 

@@ -631,6 +631,19 @@ ql_status qlinear_debug_set_fault(qlinear_t h, int32_t mode) {
   return QL_OK;
 }
 
+ql_status qlinear_debug_encode(int32_t mode, const void* in, int64_t n, const float* amax,
+                              void* out, void* stream) {
+  if (mode < 0 || mode > 2 || n < 0 || n > (int64_t{1} << 40)) return QL_ERR_INVALID_ARG;
+  if (n == 0) return QL_OK;
+  if (!in || !out || (mode == 2 && (!amax || n % 16 != 0))) return QL_ERR_INVALID_ARG;
+  if (!aligned16(in) || !aligned16(out) || (mode == 2 && (reinterpret_cast<uintptr_t>(amax) & 3)))
+    return QL_ERR_ALIGNMENT;
+  cudaError_t e = launch_debug_encode(mode, in, n, amax, static_cast<uint8_t*>(out),
+                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) cudaGetLastError();
+  return from_cuda(e);
+}
+
 ql_status qlinear_destroy(qlinear_t h) {
   if (!h) return QL_ERR_INVALID_ARG;
   delete h;

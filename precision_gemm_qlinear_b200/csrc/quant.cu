@@ -148,9 +148,8 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
   grid_dep_launch_dependents();
   if (w >= mpad) return;  // warp-uniform
   const int64_t row = mpad - 1 - w;
-  const float A = __uint_as_float(*amax_bits);
-  const float G = __fdiv_rn(A, 2688.f);
-  const float enc = A > 0.f ? __fdiv_rn(448.f, A) : 0.f;
+  float G, enc;
+  nvfp4_tensor_factors(__uint_as_float(*amax_bits), G, enc);
   if (w == 0 && lane == 0 && g_out != nullptr) *g_out = G;
   const bool live = row < M;
   const int64_t nvec = K >> 3;  // 16-byte vectors of a row
@@ -191,6 +190,35 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
       }
     }
   }
+}
+
+// ------------------------------------------------------------- test hook
+
+// The device encoders on given values, for tests that compare them with a
+// reference encoder value by value: mode 0 E4M3 and mode 1 E2M1 (one code per
+// byte) of fp32 inputs, one thread per value, through the conversions the
+// quantize kernels use; mode 2 NVFP4 16-element bf16 blocks against the
+// tensor amax *amax, one thread per block, through the block encoder of the
+// NVFP4-output GEMM epilogue (8 code bytes per block, then one scale byte
+// per block after all the codes).
+__global__ void debug_encode_kernel(int mode, const void* __restrict__ in, int64_t n,
+                                    const float* __restrict__ amax, uint8_t* __restrict__ out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (mode != 2) {
+    if (i >= n) return;
+    const float v = static_cast<const float*>(in)[i];
+    out[i] = static_cast<uint8_t>(mode == 0 ? (cvt_e4m3x2(0.f, v) & 0xFF) : (cvt_e2m1x2(0.f, v) & 0xF));
+    return;
+  }
+  const int64_t nb = n >> 4;
+  if (i >= nb) return;
+  const uint4* x = static_cast<const uint4*>(in) + 2 * i;
+  float G, enc, amb;
+  nvfp4_tensor_factors(*amax, G, enc);
+  uint2 codes;
+  const uint32_t sb = nvfp4_block(x[0], x[1], enc, G, codes, amb);
+  reinterpret_cast<uint2*>(out)[i] = codes;
+  out[8 * nb + i] = static_cast<uint8_t>(sb);
 }
 
 // ---------------------------------------------------- pre-quantized import
@@ -320,6 +348,15 @@ cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx,
   cudaLaunchConfig_t c = pdl_config(static_cast<unsigned>(blocks), 256, 0, st, at, 0);
   return cudaLaunchKernelEx(&c, quant_nvfp4_kernel<4>, static_cast<const __nv_bfloat16*>(x), M, K,
                             ldx, q, sf, sf_layout, bn, nks, mpad, amax_bits, g_out, map);
+}
+
+cudaError_t launch_debug_encode(int mode, const void* in, int64_t n, const float* amax,
+                                uint8_t* out, cudaStream_t st) {
+  const int64_t threads = mode == 2 ? (n >> 4) : n;
+  if (threads <= 0) return cudaSuccess;
+  debug_encode_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(mode, in, n,
+                                                                                     amax, out);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_qk_weights(const void* q_bf16, const void* k_bf16, float* dst,

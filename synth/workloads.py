@@ -84,6 +84,11 @@ WORKLOADS = {
     "cfg_linear1_fp8": Workload("cfg_linear1_fp8", (
         Layer("fp8", 33792, 3072, 21504, "split_bias_gelu", _T3_OUT20, split_col=9216),
     ), "CFG-batched parallel-block linear1, FP8, 33792x3072x21504, split bias/GELU"),
+    "cfg_linear1": Workload("cfg_linear1", (
+        Layer("fp8", 33792, 3072, 21504, "split_bias_gelu", _T3_OUT20, split_col=9216),
+        Layer("nvfp4", 33792, 3072, 21504, "split_bias_gelu", _T3_OUT20, split_col=9216),
+    ), "CFG-batched parallel-block linear1 in its FP8 and NVFP4 variants (two independent "
+       "layers on their own inputs), 33792x3072x21504 each, split bias/GELU"),
     "cfg_linear1_nvfp4": Workload("cfg_linear1_nvfp4", (
         Layer("nvfp4", 33792, 3072, 21504, "split_bias_gelu", _T3_OUT20, split_col=9216),
     ), "CFG-batched parallel-block linear1, NVFP4, 33792x3072x21504, split bias/GELU"),

@@ -7,7 +7,8 @@ last row, the last row and seeded random rows:
   * activation codes and scales bit for bit against the oracle's
     quantization of the same rows (NVFP4: with the whole tensor's amax, which
     numpy takes exactly from the bf16 bits);
-  * outputs within |gpu - ref| <= 8e-3 |ref| + 1e-3 rms(ref).
+  * outputs within |gpu - ref| <= 8e-3 |ref| + 1e-3 rms(ref), with rms(ref)
+    bounded from below over the whole output (see _whole_output_rms).
 A layer fed by another layer takes the GPU's bf16 output of that layer as its
 input on both sides.  The NVFP4 MLP also runs with the down projection's input
 quantized inside the up projection's epilogue.
@@ -63,6 +64,19 @@ def _check_codes(layer, d, x_bits, rows, what, amax=None):
             f"{what}: global scale"
 
 
+def _whole_output_rms(out, ref_rows):
+    """rms(ref) of the tolerance is over the whole output, which the oracle
+    cannot compute at these sizes.  Used instead: the smaller of the sampled
+    rows' rms(ref) and rms(gpu over the whole output) / 1.009 -- the least
+    rms(ref) can be when every element meets the tolerance (|gpu| <=
+    1.008 |ref| + 0.001 rms(ref)).  The smaller value is the tighter bound."""
+    import torch
+    o = out.double()
+    whole = float(torch.sqrt(torch.mean(o * o)).item())
+    sample = float(np.sqrt(np.mean(np.asarray(ref_rows, np.float64) ** 2)))
+    return min(sample, whole / 1.009)
+
+
 def _reference(layer, inp, x_bits, rows, amax=None):
     if amax is not None:
         # NVFP4 input quantized against a supplied amax: the oracle's steps
@@ -84,7 +98,7 @@ def _check_model(name, fuse=False):
     import torch
     import bench
     wl = WORKLOADS[name]
-    model = bench.Model(wl, "cuda", 0, 2 if fuse else 1, fuse=fuse)
+    model = bench.Model(wl, "cuda", 0, 2 if fuse else 1, fuse=fuse, distinct=fuse)
     layers = model.sets[0]
     supplied = {}
     if fuse:
@@ -96,9 +110,9 @@ def _check_model(name, fuse=False):
         ys = [_bits(d["out"]) for d in layers]
         supplied = {j: float(model.amax_of(model.sets[1], j).cpu()[0])
                     for j in range(1, len(layers)) if model.fused[j]}
-        model.run_layers(layers, layers[0]["x"], None, amax_from=model.sets[1])
+        model.run_layers(layers, None, amax_from=model.sets[1])
     else:
-        model.run_layers(layers, layers[0]["x"], None)
+        model.run_layers(layers, None)
     torch.cuda.synchronize()
     for li, (layer, d) in enumerate(zip(wl.layers, layers)):
         assert d["lay"].check() == 0
@@ -111,7 +125,8 @@ def _check_model(name, fuse=False):
             continue  # this layer's output went straight into the next layer's codes
         got = (_rows_of(d["out"].view(torch.int16), rows, d["out"].shape[1]).view(np.uint16)
                .astype(np.uint32) << 16).view(np.float32)
-        assert_close(got, _reference(layer, inp, x_bits, rows, supplied.get(li)), what)
+        ref = _reference(layer, inp, x_bits, rows, supplied.get(li))
+        assert_close(got, ref, what, rms=_whole_output_rms(d["out"], ref))
 
 
 @pytest.mark.parametrize("name", FULL)

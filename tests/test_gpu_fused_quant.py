@@ -4,7 +4,8 @@ quantization fused into the producing GEMM).
 The epilogue rounds each value to bf16 exactly as the bf16 path stores it and
 quantizes that with a supplied tensor amax, so:
   * with the output's true amax its codes and scales are byte-identical to the
-    standalone quantize kernel run on the bf16 output;
+    standalone quantize kernel run on the bf16 output, and bit-exact against
+    the oracle's NVFP4 quantization of that output (every epilogue);
   * with any other amax (here one that saturates) codes, block scales and G
     are bit-exact against the oracle's NVFP4 quantization of the same bf16
     values with that amax, and the recorded observed amax is max |output|.
@@ -86,6 +87,12 @@ def test_fused_output_equals_quantize_kernel_at_true_amax(epi, N, K, variant):
     assert np.array_equal(qc[: M * Nout // 2].cpu().numpy(), rc[: M * Nout // 2].cpu().numpy())
     # block scales (padding included), then G and the amax word of the tail
     assert np.array_equal(qs[: nsf + 8].cpu().numpy(), rs[: nsf + 8].cpu().numpy())
+    # and directly against the oracle's NVFP4 quantization of the bf16 output
+    oc, osf, og = oracle.quant_nvfp4(ybits)
+    sb = qs.cpu().numpy()
+    assert np.array_equal(qc[: M * Nout // 2].cpu().numpy().reshape(M, Nout // 2), oc)
+    assert np.array_equal(sf_unswizzle(sb[:nsf], M, Nout), osf)
+    assert sb[nsf:nsf + 4].view(np.uint32)[0] == np.float32(og).view(np.uint32)
 
 
 @pytest.mark.parametrize("variant", [1, 2])
