@@ -8,8 +8,6 @@
 //          mbarrier, and the leader's single MMA thread drives both tensor
 //          cores.  Per SM, 32 KB of operands feed 512 cycles of FP8 MMA.
 //   CG = 1: one CTA computes a 128 x 256 tile (used when M <= 128).
-//   The kernel can also compute two row subtiles per CTA against one
-//   128-column weight tile (Cfg::MSUB); the current configuration uses one.
 // Roles (10 warps):
 //   warp 0      TMA producer: A / B tiles (128-byte swizzle) and, for NVFP4,
 //               the block-scale atoms, into an S-stage shared-memory ring
@@ -94,15 +92,8 @@ struct Cfg {
   // Tile N: 256 (NVFP4 included: its eight scale-factor copies per stage
   // cost the same whatever N, so the widest MMA amortizes them best; the
   // two accumulators then overlap in TMEM, see below).
-  // MSUB row subtiles per CTA against one converted weight stage (tile
-  // (MSUB x 128 CG) x 128 for MSUB = 2, halving the conversion per MMA).
-  // The kernel supports 2 for weight-only layers whose epilogue does not
-  // need 256-column tiles, but one subtile with a fifth operand stage (which
-  // two subtiles leave no room for) is faster since the converted stages
-  // are published cheaply, so 1 is used throughout.
-  static constexpr int MSUB = 1;
-  static constexpr int BN = MSUB == 2 ? 128 : 256;
-  static constexpr int A_BYTES = MSUB * A_TILE_BYTES;  // this stage's rows of A
+  static constexpr int BN = 256;
+  static constexpr int A_BYTES = A_TILE_BYTES;  // this stage's rows of A
   static constexpr int B_BYTES = (BN / CG) * BK_BYTES;  // this CTA's rows of B
   static constexpr int SFA_BYTES = NV ? 2048 : 0;       // 4 atoms (one per MMA K step)
   static constexpr int SFB_BYTES = NV ? 16384 : 0;      // 4 replicated 4 KB chunks (all 256 B rows)
@@ -123,7 +114,7 @@ struct Cfg {
   // [192,256); the epilogue reads the shared columns first and releases them
   // early.
   static constexpr bool OVL = NV && BN == 256;
-  static constexpr uint32_t ACC1 = OVL ? 192 : MSUB * BN;
+  static constexpr uint32_t ACC1 = OVL ? 192 : BN;
   static constexpr uint32_t SFA_COL = 448;
   static constexpr uint32_t SFB_COL = 464;
   static_assert(!NV || ACC1 + BN <= SFA_COL, "TMEM budget");
@@ -206,24 +197,88 @@ constexpr float kGeluA = -2.302208198144325f;
 constexpr float kGeluB = -0.1029432395800235f;
 constexpr float kNegLog2e = -1.4426950408889634f;
 
-// Whole-chunk forms: each phase runs over all 32 independent elements of a
-// thread's chunk, so consecutive instructions do not depend on each other.
-__device__ __forceinline__ void gelu_tanh_32(float (&v)[32]) {
-  float d[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) d[i] = v[i] * fmaf(kGeluB, v[i] * v[i], kGeluA);
-#pragma unroll
-  for (int i = 0; i < 32; ++i) d[i] = 1.0f + ex2_sfu(d[i]);
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] *= rcp_sfu(d[i]);
+// Two fp32 values in one 64-bit register (element 0 in the low half) for the
+// packed f32x2 arithmetic of sm_100: one instruction per pair, each half
+// rounded exactly as the scalar operation (fma.rn / mul.rn / add.rn), so the
+// results equal the scalar code's bit for bit with half the instructions.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// bf16x2 word -> the pair of its two values
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
+  return f2pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
-__device__ __forceinline__ void silu_mul_32(float (&g)[32], const float (&u)[32]) {
-  float d[32];
+// GELU-tanh and SiLU on 16 pairs (the forms above, pair by pair); each phase
+// runs over all 16 independent pairs, so consecutive instructions do not
+// depend on each other.
+__device__ __forceinline__ void gelu_tanh_16x2(uint64_t (&v)[16]) {
+  const uint64_t A2 = f2pack(kGeluA, kGeluA), B2 = f2pack(kGeluB, kGeluB);
+  const uint64_t one2 = f2pack(1.f, 1.f);
+  uint64_t d[16];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) d[i] = 1.0f + ex2_sfu(kNegLog2e * g[i]);
+  for (int k = 0; k < 16; ++k) d[k] = mul2(v[k], fma2(B2, mul2(v[k], v[k]), A2));
 #pragma unroll
-  for (int i = 0; i < 32; ++i) g[i] = g[i] * rcp_sfu(d[i]) * u[i];
+  for (int k = 0; k < 16; ++k) {
+    float x0, x1;
+    f2unpack(d[k], x0, x1);
+    d[k] = add2(f2pack(ex2_sfu(x0), ex2_sfu(x1)), one2);
+  }
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    float y0, y1;
+    f2unpack(d[k], y0, y1);
+    v[k] = mul2(v[k], f2pack(rcp_sfu(y0), rcp_sfu(y1)));
+  }
+}
+
+// g <- silu(g) * u, pair by pair
+__device__ __forceinline__ void silu_mul_16x2(uint64_t (&g)[16], const uint64_t (&u)[16]) {
+  const uint64_t nl2 = f2pack(kNegLog2e, kNegLog2e), one2 = f2pack(1.f, 1.f);
+  uint64_t d[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    float x0, x1;
+    f2unpack(mul2(nl2, g[k]), x0, x1);
+    d[k] = add2(f2pack(ex2_sfu(x0), ex2_sfu(x1)), one2);
+  }
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    float y0, y1;
+    f2unpack(d[k], y0, y1);
+    g[k] = mul2(mul2(g[k], f2pack(rcp_sfu(y0), rcp_sfu(y1))), u[k]);
+  }
+}
+
+// 32 fp32 values (16 pairs) from global memory, 16 bytes per load
+__device__ __forceinline__ void load_f2x16(const float* p, uint64_t (&o)[16]) {
+  const ulonglong2* q = reinterpret_cast<const ulonglong2*>(p);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const ulonglong2 t = __ldg(q + i);
+    o[2 * i] = t.x;
+    o[2 * i + 1] = t.y;
+  }
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -231,31 +286,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// 32 bf16 kept packed (16 registers); element i is bf16x32_at(v, i).
+// 32 bf16 kept packed (16 registers).
 __device__ __forceinline__ void load_bf16x32_packed(const __nv_bfloat16* p, uint4 (&v)[4]) {
   const uint4* q = reinterpret_cast<const uint4*>(p);
 #pragma unroll
   for (int i = 0; i < 4; ++i) v[i] = __ldg(q + i);
 }
-__device__ __forceinline__ float bf16x32_at(const uint4 (&v)[4], int i) {
-  const uint4& w = v[i >> 3];
-  const int k = (i >> 1) & 3;
-  const uint32_t word = k == 0 ? w.x : (k == 1 ? w.y : (k == 2 ? w.z : w.w));
-  return (i & 1) ? bf16hi(word) : bf16lo(word);
-}
-
-__device__ __forceinline__ void load_f32x32(const float* p, float (&o)[32]) {
-  const float4* q = reinterpret_cast<const float4*>(p);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float4 v = __ldg(q + i);
-    o[4 * i] = v.x;
-    o[4 * i + 1] = v.y;
-    o[4 * i + 2] = v.z;
-    o[4 * i + 3] = v.w;
-  }
-}
-
 // OQ = 1: the epilogue writes NVFP4 codes and block scales for the next
 // layer instead of bf16 (see GemmParams::q_*).
 template <int FMT, int EPI, int CG, int OQ>
@@ -326,7 +362,7 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
       for (int t = unit; t < num_tiles && ok; t += nunits) {
         int mb, nb;
         tile_coords(t, p, mb, nb);
-        const int a_row = mb * (BM * CG * C::MSUB) + static_cast<int>(rank) * BM;  // subtile 0
+        const int a_row = mb * (BM * CG) + static_cast<int>(rank) * BM;
         const int b_row = nb * BN + static_cast<int>(rank) * (BN / CG);
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!wait_bar(&sb->empty[stage], phase ^ 1, sb, p.err, ERR_WAIT_PRODUCER)) {
@@ -348,10 +384,7 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
                 // at the leader; the raw FP8 weights on this CTA's own barrier,
                 // where this CTA's converter warps wait for them
                 if (rank == 0) mbar_arrive_expect_tx(fb, 2 * C::A_BYTES);
-#pragma unroll
-                for (int sub = 0; sub < C::MSUB; ++sub)
-                  tma_load_2d_pair(smem_u32(st + sub * A_TILE_BYTES), &p.tmA, lfb, kb * 64,
-                                   a_row + sub * BM * CG);
+                tma_load_2d_pair(smem_u32(st), &p.tmA, lfb, kb * 64, a_row);
                 const uint32_t xb = smem_u32(&sb->b8_full[stage]);
                 mbar_arrive_expect_tx(xb, C::B8_BYTES);
                 tma_load_2d(smem_u32(st + C::A_BYTES + C::B_BYTES), &p.tmB, xb, kb * 64, b_row);
@@ -374,10 +407,7 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
             } else {
               if constexpr (C::W16) {
                 mbar_arrive_expect_tx(fb, C::A_BYTES);
-#pragma unroll
-                for (int sub = 0; sub < C::MSUB; ++sub)
-                  tma_load_2d(smem_u32(st + sub * A_TILE_BYTES), &p.tmA, fb, kb * 64,
-                              a_row + sub * BM * CG);
+                tma_load_2d(smem_u32(st), &p.tmA, fb, kb * 64, a_row);
                 const uint32_t xb = smem_u32(&sb->b8_full[stage]);
                 mbar_arrive_expect_tx(xb, C::B8_BYTES);
                 tma_load_2d(smem_u32(st + C::A_BYTES + C::B_BYTES), &p.tmB, xb, kb * 64, b_row);
@@ -446,9 +476,81 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
           sdesc_k_interleave2(s0 + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, 128, 256);
       const uint32_t t_sfa = tmem + C::SFA_COL;
       const uint32_t t_sfb = tmem + C::SFB_COL;
-      for (int t = unit; t < num_tiles && ok; t += nunits, ++local) {
+      uint64_t so = 0;  // this stage's descriptor offset (16-byte units)
+      // Bring in one pipeline stage: wait for its operands (weight-only
+      // layers: and for their bf16 conversion by both CTAs), then, for
+      // NVFP4, copy its scale factors into TMEM: per MMA step j the A atom
+      // (32 x 128-bit, replicated to the 4 sub-partitions by the copy) and
+      // the pre-replicated B chunk (128 x 256-bit).  The copies do not touch
+      // the accumulator, so a tile's first stage is brought in before its
+      // accumulator is free: the tensor pipe runs those copies while the
+      // epilogue still drains the previous tile.
+      auto stage_in = [&]() -> bool {
+        if (!wait_bar(&sb->full[stage], phase, sb, p.err, ERR_WAIT_MMA)) return false;
+        if constexpr (C::W16) {
+          if (!wait_bar<true>(&sb->conv_done[stage], phase, sb, p.err, ERR_WAIT_MMA)) return false;
+        }
+        tc_fence_after();
+        // the stage-0 descriptors advanced by the stage offset in the
+        // 16-byte start-address field
+        so = static_cast<uint64_t>(stage) * (C::STAGE_BYTES >> 4);
+        if constexpr (C::NV) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t da = d_sfa0 + so + (512 >> 4) * j;
+            const uint64_t db = d_sfb0 + so + (4096 >> 4) * j;
+            if constexpr (C::PAIR) {
+              tc_cp_32x128b_warpx4_pair(t_sfa + 4 * j, da);
+              tc_cp_128x256b_pair(t_sfb + 8 * j, db);
+            } else {
+              tc_cp_32x128b_warpx4(t_sfa + 4 * j, da);
+              tc_cp_128x256b(t_sfb + 8 * j, db);
+            }
+          }
+          any = true;
+        }
+        return true;
+      };
+      // The stage's four MMA steps (K = 64 FP4 / 32 FP8 / 16 bf16 elements
+      // each, 32 bytes of every operand row), then release the stage.
+      auto stage_mma = [&](uint32_t d_tmem, bool first) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint64_t ad = d_a0 + so + (32 >> 4) * j;
+          const uint64_t bd = d_b0 + so + (32 >> 4) * j;
+          const uint32_t acc = (!first || j > 0) ? 1u : 0u;
+          if constexpr (C::NV) {
+            if constexpr (C::PAIR)
+              mma_mxf4nvf4_pair(d_tmem, ad, bd, idesc_f4<CG, BN>(), t_sfa + 4 * j, t_sfb + 8 * j,
+                                acc);
+            else
+              mma_mxf4nvf4(d_tmem, ad, bd, idesc_f4<CG, BN>(), t_sfa + 4 * j, t_sfb + 8 * j, acc);
+          } else if constexpr (C::W16) {
+            if constexpr (C::PAIR)
+              mma_bf16_pair(d_tmem, ad, bd, idesc_bf16<CG, BN>(), acc);
+            else
+              mma_bf16(d_tmem, ad, bd, idesc_bf16<CG, BN>(), acc);
+          } else {
+            if constexpr (C::PAIR)
+              mma_f8f6f4_pair(d_tmem, ad, bd, idesc_f8<CG, BN>(), acc);
+            else
+              mma_f8f6f4(d_tmem, ad, bd, idesc_f8<CG, BN>(), acc);
+          }
+        }
+        any = true;
+        if constexpr (C::PAIR)
+          tc_commit_pair_mc(smem_u32(&sb->empty[stage]), 0x3);
+        else
+          tc_commit(smem_u32(&sb->empty[stage]));
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      };
+      for (int t = unit; t < num_tiles; t += nunits, ++local) {
         const int buf = local & 1;
         const uint32_t use = static_cast<uint32_t>(local >> 1);
+        if (!stage_in()) break;
         if (!wait_bar(&sb->acc_empty[buf], (use & 1) ^ 1, sb, p.err, ERR_WAIT_MMA)) break;
         if (C::OVL && local > 0 &&
             !wait_bar(&sb->ovl_free, static_cast<uint32_t>(local - 1) & 1, sb, p.err,
@@ -456,77 +558,13 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
           break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + (buf ? C::ACC1 : 0u);
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
-          if (!wait_bar(&sb->full[stage], phase, sb, p.err, ERR_WAIT_MMA)) {
+        stage_mma(d_tmem, true);
+        for (int kb = 1; kb < p.k_blocks; ++kb) {
+          if (!stage_in()) {
             ok = false;
             break;
           }
-          if constexpr (C::W16) {
-            // both CTAs' converter warps have written this stage's bf16 B
-            if (!wait_bar<true>(&sb->conv_done[stage], phase, sb, p.err, ERR_WAIT_MMA)) {
-              ok = false;
-              break;
-            }
-          }
-          tc_fence_after();
-          // this stage's descriptors: the stage-0 descriptors advanced by the
-          // stage offset in the 16-byte start-address field
-          const uint64_t so = static_cast<uint64_t>(stage) * (C::STAGE_BYTES >> 4);
-          if constexpr (C::NV) {
-            // per MMA step j: the A atom (32 x 128-bit, replicated to the 4
-            // sub-partitions by the copy) and the pre-replicated B chunk
-            // (128 x 256-bit)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint64_t da = d_sfa0 + so + (512 >> 4) * j;
-              const uint64_t db = d_sfb0 + so + (4096 >> 4) * j;
-              if constexpr (C::PAIR) {
-                tc_cp_32x128b_warpx4_pair(t_sfa + 4 * j, da);
-                tc_cp_128x256b_pair(t_sfb + 8 * j, db);
-              } else {
-                tc_cp_32x128b_warpx4(t_sfa + 4 * j, da);
-                tc_cp_128x256b(t_sfb + 8 * j, db);
-              }
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint64_t ad = d_a0 + so + (32 >> 4) * j;
-            const uint64_t bd = d_b0 + so + (32 >> 4) * j;
-            const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
-            if constexpr (C::NV) {
-              if constexpr (C::PAIR)
-                mma_mxf4nvf4_pair(d_tmem, ad, bd, idesc_f4<CG, BN>(), t_sfa + 4 * j, t_sfb + 8 * j,
-                                  acc);
-              else
-                mma_mxf4nvf4(d_tmem, ad, bd, idesc_f4<CG, BN>(), t_sfa + 4 * j, t_sfb + 8 * j,
-                             acc);
-            } else if constexpr (C::W16) {
-              // one MMA per row subtile, all against the same B stage
-#pragma unroll
-              for (int sub = 0; sub < C::MSUB; ++sub) {
-                const uint64_t as = ad + sub * (A_TILE_BYTES >> 4);
-                if constexpr (C::PAIR)
-                  mma_bf16_pair(d_tmem + sub * BN, as, bd, idesc_bf16<CG, BN>(), acc);
-                else
-                  mma_bf16(d_tmem + sub * BN, as, bd, idesc_bf16<CG, BN>(), acc);
-              }
-            } else {
-              if constexpr (C::PAIR)
-                mma_f8f6f4_pair(d_tmem, ad, bd, idesc_f8<CG, BN>(), acc);
-              else
-                mma_f8f6f4(d_tmem, ad, bd, idesc_f8<CG, BN>(), acc);
-            }
-          }
-          any = true;
-          if constexpr (C::PAIR)
-            tc_commit_pair_mc(smem_u32(&sb->empty[stage]), 0x3);
-          else
-            tc_commit(smem_u32(&sb->empty[stage]));
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1;
-          }
+          stage_mma(d_tmem, false);
         }
         if (!ok) break;
         if constexpr (C::PAIR)
@@ -623,7 +661,6 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
     uint8_t* staging = smem + C::STAGING_OFF + ew * C::NBUF * STAGING_BYTES;
     // 32-column output chunks per tile
     constexpr int NCHT = (EPI == EPI_SWIGLU) ? BN / 64 : BN / 32;
-    constexpr bool MS = C::MSUB == 2;
     const uint32_t ovl_l0 = mapa_shared(smem_u32(&sb->ovl_free), 0);
     int local = 0;
     uint32_t nstore = 0;
@@ -643,16 +680,14 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
       tc_fence_after();
       // Each sub-partition's work is split in two halves: with eight
       // epilogue warps the two warps of a sub-partition take one each, with
-      // four each warp takes both, one per pass.  A half is the row subtile
-      // (two subtiles per CTA), else alternate 32-column chunks (the head,
-      // for QKV).  Every (warp, pass) releases the accumulator once.
+      // four each warp takes both, one per pass.  A half is alternate
+      // 32-column chunks (the head, for QKV).  Every (warp, pass) releases
+      // the accumulator once.
 #pragma unroll 1
       for (int pass = 0; pass < C::EPI_PASSES; ++pass) {
         const int half = C::EPI_PASSES == 2 ? pass : (ew >> 2);
-        const int nch = MS ? NCHT : (NCHT - half + 1) >> 1;  // this half's chunks
-        const int sub = MS ? half : 0;  // row subtile of this warp
-        const int row0 = mb * (BM * CG * C::MSUB) + sub * (BM * CG) + static_cast<int>(rank) * BM +
-                         sp * 32;  // first row of this warp
+        const int nch = (NCHT - half + 1) >> 1;  // this half's chunks
+        const int row0 = mb * (BM * CG) + static_cast<int>(rank) * BM + sp * 32;  // first row of this warp
         const int m = row0 + lane;
         const bool row_ok = m < p.M;
         const bool slab_ok = row0 < p.M;
@@ -663,8 +698,7 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
           rs = 1.f;  // bf16 activations carry no scale
         else
           rs = row_ok ? __ldg(p.sa + m) : 0.f;
-        const uint32_t tbase = tmem + (static_cast<uint32_t>(sp * 32) << 16) + (buf ? C::ACC1 : 0u) +
-                               static_cast<uint32_t>(sub * BN);
+        const uint32_t tbase = tmem + (static_cast<uint32_t>(sp * 32) << 16) + (buf ? C::ACC1 : 0u);
         // one 32 x 32 bf16 box: swizzled shared staging, then a TMA store
         auto store_chunk = [&](const uint32_t (&pk)[16], int ocol) {
           uint8_t* sbuf = staging + (nstore % C::NBUF) * STAGING_BYTES;
@@ -696,22 +730,24 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
           const float* wgt = p.qk_w + (h0 < p.k_col0 ? 0 : QKV_HEAD_DIM);
           const int64_t mrow = row_ok ? m : p.M - 1;  // padded rows read row M-1's angles
           auto values = [&](int k, const uint32_t (&a)[32], float (&v)[32]) {
-            uint4 bp[4];
-            load_bf16x32_packed(p.bias + h0 + 32 * k, bp);
-            if constexpr (C::NV) {
+            const float4* bp = reinterpret_cast<const float4*>(p.bias + h0 + 32 * k);
+            const float4* swp = reinterpret_cast<const float4*>(p.sw + h0 + 32 * k);
   #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = fmaf(__uint_as_float(a[i]), rs, bf16x32_at(bp, i));
-            } else {
-              const float4* swp = reinterpret_cast<const float4*>(p.sw + h0 + 32 * k);
-  #pragma unroll
-              for (int i4 = 0; i4 < 8; ++i4) {
+            for (int i4 = 0; i4 < 8; ++i4) {
+              const float4 b4 = __ldg(bp + i4);
+              const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+              float sw4[4] = {1.f, 1.f, 1.f, 1.f};
+              if constexpr (!C::NV) {
                 const float4 s4 = __ldg(swp + i4);
-                const float sw4[4] = {s4.x, s4.y, s4.z, s4.w};
+                sw4[0] = s4.x;
+                sw4[1] = s4.y;
+                sw4[2] = s4.z;
+                sw4[3] = s4.w;
+              }
   #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  const int i = 4 * i4 + j;
-                  v[i] = fmaf(__uint_as_float(a[i]), rs * sw4[j], bf16x32_at(bp, i));
-                }
+              for (int j = 0; j < 4; ++j) {
+                const int i = 4 * i4 + j;
+                v[i] = fmaf(__uint_as_float(a[i]), C::NV ? rs : rs * sw4[j], bb[j]);
               }
             }
           };
@@ -791,11 +827,10 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
         // the gate half of chunks 0, 1 in buffer 1; every warp holds exactly one
         // of them and reads it first.
         auto chunk_of = [&](int ci) {
-          if (MS) return ci;
           const int k = (C::OVL && buf == 0) ? (nch - 1 - ci) : ci;
           return half + 2 * k;
         };
-        constexpr int NCHW = MS ? NCHT : (NCHT + 1) / 2;  // most chunks a warp can have
+        constexpr int NCHW = (NCHT + 1) / 2;  // most chunks a warp can have
         uint32_t acc[2][32];                   // double-buffered accumulator chunk
         uint32_t accu[32];                     // SwiGLU: the up half
         tmem_ld_32x32b_x32(tbase + 32 * chunk_of(0), acc[0]);
@@ -810,14 +845,10 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
           const bool live = ncol < p.N;  // past the last column (N % 32 == 0); warp-uniform
           // per-column and per-row operands: issued before the TMEM wait so the
           // two latencies overlap
-          uint4 bias_a[4], bias_b[4], gate_a[4], res_a[4];
-          float sw_a[32];
+          uint64_t bias2[16];  // the chunk's 32 bias values as pairs
+          uint4 gate_a[4], res_a[4];
           if (live) {
-            load_bf16x32_packed(p.bias + ncol, bias_a);
-            if constexpr (!C::NV) load_f32x32(p.sw + ncol, sw_a);
-            if constexpr (EPI == EPI_SWIGLU) {
-              load_bf16x32_packed(p.bias + ncol + 128, bias_b);
-            }
+            load_f2x16(p.bias + ncol, bias2);
             if constexpr (EPI == EPI_GATED_RES) {
               // per-batch gates (CFG-batched tokens): row m uses gate row m / gate_rows
               const __nv_bfloat16* gp = p.gate + ocol;
@@ -850,51 +881,66 @@ __global__ void __launch_bounds__(Cfg<FMT, CG, EPI>::THREADS, 1)
           const uint32_t* ra = acc[(EPI == EPI_SWIGLU) ? 0 : (ci & 1)];
           uint32_t packed[16];
           if (live) {
-            float v[32];
-            if constexpr (EPI == EPI_SWIGLU) {
-              float u[32];
-              // FP8: the up half's column scales are read in float4 pieces here
-              // (two preloaded 32-float arrays would not fit in registers)
-              const float4* swb = reinterpret_cast<const float4*>(p.sw + ncol + 128);
+            // y = acc * scale + bias, pair by pair (FP8: scale = s_a[m] * s_w[n];
+            // NVFP4: G_a * G_w)
+            const uint64_t rs2 = f2pack(rs, rs);
+            uint64_t v2[16];
+            if constexpr (C::NV) {
   #pragma unroll
-              for (int i4 = 0; i4 < 8; ++i4) {
-                float sb4[4] = {rs, rs, rs, rs};
-                if constexpr (!C::NV) {
-                  const float4 w4 = __ldg(swb + i4);
-                  sb4[0] = rs * w4.x;
-                  sb4[1] = rs * w4.y;
-                  sb4[2] = rs * w4.z;
-                  sb4[3] = rs * w4.w;
-                }
-  #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  const int i = 4 * i4 + j;
-                  const float sa_ = C::NV ? rs : rs * sw_a[i];
-                  v[i] = fmaf(__uint_as_float(ra[i]), sa_, bf16x32_at(bias_a, i));
-                  u[i] = fmaf(__uint_as_float(accu[i]), sb4[j], bf16x32_at(bias_b, i));
-                }
-              }
-              silu_mul_32(v, u);
+              for (int k = 0; k < 16; ++k)
+                v2[k] = fma2(f2pack(__uint_as_float(ra[2 * k]), __uint_as_float(ra[2 * k + 1])), rs2,
+                             bias2[k]);
             } else {
+              uint64_t sw2[16];
+              load_f2x16(p.sw + ncol, sw2);
   #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                float s_;
-                if constexpr (C::NV)
-                  s_ = rs;
-                else
-                  s_ = rs * sw_a[i];
-                v[i] = fmaf(__uint_as_float(ra[i]), s_, bf16x32_at(bias_a, i));
-                if constexpr (EPI == EPI_GATED_RES)
-                  v[i] = fmaf(bf16x32_at(gate_a, i), v[i], bf16x32_at(res_a, i));
+              for (int k = 0; k < 16; ++k)
+                v2[k] = fma2(f2pack(__uint_as_float(ra[2 * k]), __uint_as_float(ra[2 * k + 1])),
+                             mul2(rs2, sw2[k]), bias2[k]);
+            }
+            if constexpr (EPI == EPI_SWIGLU) {
+              // the up half (columns ncol + 128 ..): its bias (and FP8 column
+              // scales) are read here, after the gate half's are consumed
+              uint64_t u2[16], t2[16];
+              load_f2x16(p.bias + ncol + 128, t2);
+              if constexpr (C::NV) {
+  #pragma unroll
+                for (int k = 0; k < 16; ++k)
+                  u2[k] = fma2(f2pack(__uint_as_float(accu[2 * k]), __uint_as_float(accu[2 * k + 1])),
+                               rs2, t2[k]);
+              } else {
+                uint64_t sw2[16];
+                load_f2x16(p.sw + ncol + 128, sw2);
+  #pragma unroll
+                for (int k = 0; k < 16; ++k)
+                  u2[k] = fma2(f2pack(__uint_as_float(accu[2 * k]), __uint_as_float(accu[2 * k + 1])),
+                               mul2(rs2, sw2[k]), t2[k]);
+              }
+              silu_mul_16x2(v2, u2);
+            } else {
+              if constexpr (EPI == EPI_GATED_RES) {
+  #pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                  const uint4& gw = gate_a[k >> 2];
+                  const uint4& rw = res_a[k >> 2];
+                  const int q = k & 3;
+                  const uint32_t g = q == 0 ? gw.x : (q == 1 ? gw.y : (q == 2 ? gw.z : gw.w));
+                  const uint32_t r = q == 0 ? rw.x : (q == 1 ? rw.y : (q == 2 ? rw.z : rw.w));
+                  v2[k] = fma2(bf16x2_to_f2(g), v2[k], bf16x2_to_f2(r));
+                }
               }
               if constexpr (EPI == EPI_BIAS_GELU) {
-                gelu_tanh_32(v);
+                gelu_tanh_16x2(v2);
               } else if constexpr (EPI == EPI_SPLIT) {
-                if (ncol >= p.split_col) gelu_tanh_32(v);  // uniform per chunk
+                if (ncol >= p.split_col) gelu_tanh_16x2(v2);  // uniform per chunk
               }
             }
   #pragma unroll
-            for (int i = 0; i < 32; i += 2) packed[i >> 1] = pack_bf16x2(v[i], v[i + 1]);
+            for (int k = 0; k < 16; ++k) {
+              float lo, hi;
+              f2unpack(v2[k], lo, hi);
+              packed[k] = pack_bf16x2(lo, hi);
+            }
           }
           if constexpr (EPI == EPI_SWIGLU) {
             // SwiGLU holds two halves per chunk; the next pair is loaded here,
@@ -1006,11 +1052,6 @@ int gemm_tile_n(int fmt, int epi) {
   if (epi == EPI_SWIGLU) return Cfg<1, 2, EPI_SWIGLU>::BN;
   if (epi == EPI_QKV) return Cfg<1, 2, EPI_QKV>::BN;
   return Cfg<1, 2, EPI_BIAS>::BN;
-}
-
-int gemm_tile_msub(int fmt, int epi) {
-  if (fmt == 2 && epi != EPI_SWIGLU && epi != EPI_QKV) return Cfg<2, 2, EPI_BIAS>::MSUB;
-  return 1;
 }
 
 cudaError_t launch_gemm(int fmt, int epi, int cg, int outq, const GemmParams& p, int num_sms,

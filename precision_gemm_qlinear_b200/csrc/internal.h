@@ -106,7 +106,8 @@ cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx,
 // the block scales).
 cudaError_t launch_debug_encode(int mode, const void* in, int64_t n, const float* amax,
                                 uint8_t* out, cudaStream_t st);
-cudaError_t launch_permute_bias(const void* src, void* dst, int64_t N, RowMap map,
+// bf16 bias [N] (or null = zeros) -> fp32 [N] in the GEMM's row order.
+cudaError_t launch_permute_bias(const void* src, float* dst, int64_t N, RowMap map,
                                 cudaStream_t st);
 
 // ------------------------------------------------------------------ GEMM
@@ -130,7 +131,7 @@ struct alignas(64) GemmParams {
   const uint8_t* sfb;     // NVFP4: weight SF chunks (sfb_word_offset layout)
   const float* ga;        // NVFP4: activation global scale (device scalar)
   const float* gw;        // NVFP4: weight global scale (device scalar)
-  const __nv_bfloat16* bias;      // [N] (zeros when the layer has no bias)
+  const float* bias;              // fp32 [N] (zeros when the layer has no bias)
   const __nv_bfloat16* residual;  // [M, Nout] or null
   const __nv_bfloat16* gate;      // [Nout] or null
   __nv_bfloat16* out;             // [M, Nout] (the TMA store map tmC covers the same buffer)
@@ -167,10 +168,6 @@ cudaError_t launch_gemm(int fmt, int epi, int cg, int outq, const GemmParams& p,
                         cudaStream_t st);
 // N of the GEMM tile for a format / epilogue (the weight scale layout uses it).
 int gemm_tile_n(int fmt, int epi);
-// Row subtiles per CTA (the kernel supports 2 for weight-only layers with
-// 128-column tiles; every configuration in use has 1): a tile covers
-// 128 * cg * msub rows.
-int gemm_tile_msub(int fmt, int epi);
 
 // Error codes written to the device error word by the GEMM watchdog.
 enum : uint32_t { ERR_WAIT_PRODUCER = 1u, ERR_WAIT_MMA = 2u, ERR_WAIT_EPI = 4u };

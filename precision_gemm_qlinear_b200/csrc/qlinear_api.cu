@@ -35,12 +35,12 @@ struct qlinear_s {
   uint8_t* wsf;      // NVFP4 scale-factor atoms
   float* wG;         // NVFP4 global scale (device scalar)
   uint32_t* wamax;   // NVFP4 amax word used while quantizing W
-  __nv_bfloat16* bias;
+  float* bias;       // fp32 [N] in the GEMM's row order
   float* qk_w;         // QKV epilogue: fp32 norm weights [2][128] (q, then k)
   float qk_eps;        // QKV epilogue: RMS normalization epsilon
   RowMap map;
   int32_t fault_mode;  // test hook, see qlinear_debug_set_fault
-  int32_t bn;          // N of the GEMM tile (256, or 128 for weight-only bias-type layers)
+  int32_t bn;          // N of the GEMM tile (256)
   CUtensorMap tmB1;    // weight codes, box 128 B x 256 rows (one CTA per tile)
   CUtensorMap tmB2;    // weight codes, box 128 B x 128 rows (CTA pair per tile)
   CUtensorMap tmSFB;   // NVFP4: weight SF atoms as 2048-byte rows (CTA pair)
@@ -58,7 +58,7 @@ struct WsLayout {
   size_t err, codes, scales, bias, qk, total;
 };
 
-// Weight workspace: [control 256 B][codes][scales (+16 B tail for NVFP4)][bias]
+// Weight workspace: [control 1 KB][codes][scales (+16 B tail for NVFP4)][fp32 bias]
 WsLayout ws_layout(const ql_desc& d) {
   WsLayout L;
   L.err = 0;
@@ -73,7 +73,7 @@ WsLayout ws_layout(const ql_desc& d) {
                                             : static_cast<size_t>(d.N) * 4;
   off = align_up(off + sc_bytes, 1024);
   L.bias = off;
-  off = align_up(off + static_cast<size_t>(d.N) * 2, 1024);
+  off = align_up(off + static_cast<size_t>(d.N) * 4, 1024);
   L.qk = off;  // QKV epilogue: q and k norm weights (fp32, 2 x 128)
   if (d.epi == QL_EPI_QKV_NORM_ROPE) off += 1024;
   L.total = off;
@@ -265,7 +265,7 @@ ql_status forward_impl(qlinear_t h, const void* codes, const void* scales, int64
   p.Nout = static_cast<int32_t>(h->Nout);
   p.split_col = static_cast<int32_t>(h->d.split_col);
   p.k_blocks = static_cast<int32_t>((kbytes + 127) / 128);
-  const int64_t tile_rows = 128 * cg * gemm_tile_msub(h->d.fmt, h->d.epi);
+  const int64_t tile_rows = 128 * cg;
   p.tiles_m = static_cast<int32_t>((M + tile_rows - 1) / tile_rows);
   p.tiles_n = static_cast<int32_t>((h->N + h->bn - 1) / h->bn);
   p.group_m = 8;
@@ -333,7 +333,7 @@ ql_status begin_create(const ql_desc* desc, const void* bias_bf16, void* weight_
   h->ws_bytes = ws_bytes;
   h->err = reinterpret_cast<uint32_t*>(h->ws + L.err);
   h->wcodes = h->ws + L.codes;
-  h->bias = reinterpret_cast<__nv_bfloat16*>(h->ws + L.bias);
+  h->bias = reinterpret_cast<float*>(h->ws + L.bias);
   h->qk_w = reinterpret_cast<float*>(h->ws + L.qk);
   h->qk_eps = 1e-6f;
   h->map.nout = h->Nout;

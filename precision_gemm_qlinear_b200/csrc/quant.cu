@@ -270,10 +270,12 @@ __global__ void qk_weights_kernel(const __nv_bfloat16* __restrict__ qw,
   dst[i] = src ? __bfloat162float(src[j]) : 1.0f;
 }
 
-__global__ void permute_bias_kernel(const __nv_bfloat16* __restrict__ src,
-                                    __nv_bfloat16* __restrict__ dst, int64_t N, RowMap map) {
+// The bias widened to fp32 (exact) in the GEMM's row order, so the epilogue
+// adds it without unpacking bf16.
+__global__ void permute_bias_kernel(const __nv_bfloat16* __restrict__ src, float* __restrict__ dst,
+                                    int64_t N, RowMap map) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i < N) dst[i] = src ? src[map(i)] : __float2bfloat16(0.f);
+  if (i < N) dst[i] = src ? __bfloat162float(src[map(i)]) : 0.f;
 }
 
 }  // namespace
@@ -366,11 +368,11 @@ cudaError_t launch_qk_weights(const void* q_bf16, const void* k_bf16, float* dst
   return cudaGetLastError();
 }
 
-cudaError_t launch_permute_bias(const void* src, void* dst, int64_t N, RowMap map,
+cudaError_t launch_permute_bias(const void* src, float* dst, int64_t N, RowMap map,
                                 cudaStream_t st) {
   if (N <= 0) return cudaSuccess;
   permute_bias_kernel<<<static_cast<unsigned>((N + 255) / 256), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(src), static_cast<__nv_bfloat16*>(dst), N, map);
+      static_cast<const __nv_bfloat16*>(src), dst, N, map);
   return cudaGetLastError();
 }
 
