@@ -104,12 +104,19 @@ typedef struct {
  * a small control block).  Host only, no CUDA call. */
 QL_API ql_status qlinear_weight_bytes(const ql_desc* desc, size_t* bytes);
 
-/* Quantize W once and lay it out for the GEMM.
+/* Quantize W once and lay it out for the GEMM -- the weight half of the
+ * dynamic quantization ("Cuantizacion Dinamica FP8", wavespeed.ai "Solucion de
+ * WaveSpeed...": weights and activations both lowered to FP8; bytechap.com
+ * "Como funciona": NVFP4 lowers weights as well as activations).
  *   w_bf16    : device, [N, K] bf16 master weights (read only during the call's
  *               kernels; may be freed once the stream has passed them).
  *   bias_bf16 : device, [N] bf16, or NULL for zero bias.  Copied into weight_ws.
  *   weight_ws : device, >= qlinear_weight_bytes(desc), 256-byte aligned; must
  *               stay alive and untouched until qlinear_destroy.
+ *   ws_bytes  : the size of weight_ws, checked against qlinear_weight_bytes
+ *               (QL_ERR_INVALID_ARG if smaller) -- an argument beyond the
+ *               three-call outline of the path, so that a short buffer is an
+ *               error instead of an out-of-bounds write.
  *   stream    : the kernels are enqueued here; the handle may be used on any
  *               stream ordered after this one.
  *   out       : receives the handle (host object owned by the library).
@@ -149,7 +156,10 @@ QL_API ql_status qlinear_act_bytes(qlinear_t h, int64_t M, size_t* code_bytes, s
 /* Number of output columns of qlinear_forward (N, or N/2 for SwiGLU). */
 QL_API ql_status qlinear_out_features(qlinear_t h, int64_t* nout);
 
-/* Dynamic activation quantization (no host sync, no allocation).
+/* Dynamic activation quantization (no host sync, no allocation): the scales
+ * are computed from this call's activations ("Cuantizacion Dinamica FP8",
+ * wavespeed.ai "Solucion de WaveSpeed...": scales found at run time;
+ * algoritmulzilei.ro FLUX 3 Image Klein page: NVFP4 activations).
  *   x_bf16 : device [M, K] bf16;  codes, scales: device, sized by
  *   qlinear_act_bytes.  FP8: one fused pass (row amax, scale, cast).
  *   NVFP4: a tensor-amax pass, then the block quantize that also writes the
@@ -169,13 +179,17 @@ QL_API ql_status qlinear_quantize_act(qlinear_t h, const void* x_bf16, int64_t M
  *   Arguments and outputs are those of qlinear_quantize_act (the caller still
  *   provides x, codes and scales, sized by qlinear_act_bytes).  FP8 layers use
  *   the same single-pass kernel, which needs no working memory.  For NVFP4
- *   the working memory of the tensor-amax reduction (one partial maximum per
- *   128-row block, then the tensor maximum) is a fixed array inside the
+ *   the working memory of the tensor-amax reduction (the partial maxima of a
+ *   grid-stride pass, then the tensor maximum) is a fixed array inside the
  *   library (QL_NOALLOC_MAX_ROWS / 128 + 64 words per device, held until the
  *   process exits) instead of the amax word in the scales tail.
  *   M > QL_NOALLOC_MAX_ROWS returns QL_ERR_INVALID_ARG before any launch.
  *   The first call on a device looks up that array's device address (no
- *   allocation); make that first call before any stream capture.
+ *   allocation) and keeps it for the life of the process; make that first
+ *   call before any stream capture.  Device ordinals 64 and above return
+ *   QL_ERR_UNSUPPORTED.  The kept address does not survive a reset of the
+ *   device's primary context (cudaDeviceReset): do not call this entry
+ *   point again in a process after such a reset.
  *   All calls on a device share the array and it keeps the last call's
  *   contents; no entry of it needs to start at zero, because every call
  *   writes the entries it reads.  Calls whose kernels overlap on the GPU
@@ -184,7 +198,10 @@ QL_API ql_status qlinear_quantize_act(qlinear_t h, const void* x_bf16, int64_t M
 QL_API ql_status qlinear_quantize_act_noalloc(qlinear_t h, const void* x_bf16, int64_t M,
                                               void* codes, void* scales, void* stream);
 
-/* GEMM + fused epilogue (no host sync, no allocation).
+/* GEMM + fused epilogue (no host sync, no allocation): the matmul on the 8-bit
+ * / 4-bit tensor cores ("Cuantizacion Dinamica FP8", wavespeed.ai "Solucion de
+ * WaveSpeed...") with the epilogue fused into the GEMM (algoritmulzilei.ro
+ * FLUX 3 Image Klein page: GEMMs with fused epilogues, SwiGLU among them).
  *   codes, scales : as written by qlinear_quantize_act for the same M.
  *   residual      : device [M, Nout] bf16 for QL_EPI_BIAS_GATED_RESIDUAL, else NULL.
  *   gate          : device [Nout] bf16 for QL_EPI_BIAS_GATED_RESIDUAL, else NULL.

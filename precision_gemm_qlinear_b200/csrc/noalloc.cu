@@ -4,7 +4,7 @@
 // inside another framework's memory pool, a plugin that is handed only the
 // tensors of one operator, or a CUDA-graph replay path that must not touch
 // the allocator.  qlinear_quantize_act_noalloc serves them.  For NVFP4 its
-// only working memory (one partial amax per 128-row block and the tensor
+// only working memory (the partial maxima of the amax pass and the tensor
 // amax) lives in a file-scope device array that is part of this library, so
 // the caller passes nothing but the input and the two output buffers.
 //
@@ -25,18 +25,23 @@ namespace qlb {
 
 namespace {
 
-// Maximum number of 128-row blocks of one call (M <= 128 * 4096 = 524288 tokens).
-constexpr int kMaxRowBlocks = QL_NOALLOC_MAX_ROWS / 128;
+// Number of partial maxima the array holds (the amax pass runs at most this
+// many CTAs); M <= QL_NOALLOC_MAX_ROWS keeps every call's scales tail and
+// sizes within what the rest of the library checks.
+constexpr int kMaxPartials = QL_NOALLOC_MAX_ROWS / 128;
 
-// [0, kMaxRowBlocks): partial amax bits per row block; [kMaxRowBlocks]: tensor amax.
-static __device__ __align__(256) uint32_t g_noalloc_scratch[kMaxRowBlocks + 64];
+// [0, kMaxPartials): partial amax bits, one per CTA of the amax pass;
+// [kMaxPartials]: tensor amax.
+static __device__ __align__(256) uint32_t g_noalloc_scratch[kMaxPartials + 64];
 
 // Device address of g_noalloc_scratch per device, found once per device with
 // that device current (the array's name in host code is only a stand-in).
+// Devices 0..63 are cached; the caller rejects higher ordinals.
+constexpr int kMaxDevices = 64;
 uint32_t* scratch_ptr(int dev) {
   static std::mutex mu;
-  static uint32_t* ptrs[64] = {nullptr};
-  if (dev < 0 || dev >= 64) return nullptr;
+  static uint32_t* ptrs[kMaxDevices] = {nullptr};
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
   if (ptrs[dev] == nullptr) {
     void* p = nullptr;
@@ -57,17 +62,17 @@ __device__ __forceinline__ float absmax8_bits(const uint4& v) {
   return m;
 }
 
-// One CTA per 128-row block: max |x| over the block, written (not
-// accumulated) to partial[blockIdx.x].
-__global__ void __launch_bounds__(256) rowblock_amax_kernel(const __nv_bfloat16* __restrict__ x,
-                                                            int64_t M, int64_t K,
-                                                            uint32_t* __restrict__ partial) {
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * 128;
-  const int64_t rows = (M - r0) < 128 ? (M - r0) : 128;
-  const int64_t nvec = rows * K / 8;
-  const uint4* xv = reinterpret_cast<const uint4*>(x + r0 * K);
+// Grid-stride max |x| over the whole tensor (M * K / 8 vectors of 8): each
+// CTA writes (does not accumulate) its maximum to partial[blockIdx.x], so no
+// entry has to start at zero.
+__global__ void __launch_bounds__(256) partial_amax_kernel(const uint4* __restrict__ xv,
+                                                           int64_t nvec,
+                                                           uint32_t* __restrict__ partial) {
   float m = 0.f;
-  for (int64_t i = threadIdx.x; i < nvec; i += blockDim.x) m = fmaxf(m, absmax8_bits(__ldg(xv + i)));
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nvec;
+       i += stride)
+    m = fmaxf(m, absmax8_bits(__ldg(xv + i)));
   uint32_t a = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
   __shared__ uint32_t red[8];
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
@@ -124,18 +129,30 @@ ql_status quantize_act_noalloc(int fmt, int64_t K, int num_sms, const void* x, i
     cudaGetLastError();
     return QL_ERR_CUDA;
   }
+  if (dev >= kMaxDevices) return QL_ERR_UNSUPPORTED;
   uint32_t* scratch = scratch_ptr(dev);
   if (scratch == nullptr) return QL_ERR_CUDA;
-  const int nrb = static_cast<int>((M + 127) / 128);
+  // amax pass: up to eight CTAs an SM (never more than the array's partials),
+  // grid-stride over the tensor
+  const int64_t nvec = M * K / 8;
+  int64_t nblk = (nvec + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8 < kMaxPartials
+                          ? static_cast<int64_t>(num_sms) * 8
+                          : static_cast<int64_t>(kMaxPartials);
+  if (nblk > cap) nblk = cap;
   uint8_t* sf = static_cast<uint8_t*>(scales);
   float* g = reinterpret_cast<float*>(sf + sf_bytes(M, K));
-  rowblock_amax_kernel<<<nrb, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), M, K, scratch);
-  reduce_amax_kernel<<<1, 256, 0, st>>>(scratch, nrb, scratch + kMaxRowBlocks);
+  // Plain launches on purpose (no programmatic overlap): this call
+  // overwrites the tensor amax that the quantize kernel of a previous call on
+  // the stream reads, so these kernels may only start once that kernel has
+  // finished.
+  partial_amax_kernel<<<static_cast<unsigned>(nblk), 256, 0, st>>>(static_cast<const uint4*>(x),
+                                                                   nvec, scratch);
+  reduce_amax_kernel<<<1, 256, 0, st>>>(scratch, static_cast<int>(nblk), scratch + kMaxPartials);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess)
     e = launch_quant_nvfp4(x, M, K, K, static_cast<uint8_t*>(codes), sf, 0, 128,
-                           scratch + kMaxRowBlocks,
-                           g, RowMap{0, 0}, st);
+                           scratch + kMaxPartials, g, RowMap{0, 0}, st);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return QL_ERR_CUDA;

@@ -71,6 +71,39 @@ def test_noalloc_matches_quantize_act_twice_in_a_row(fmt):
     lay.close()
 
 
+@pytest.mark.parametrize("M,K", [(4608, 3072), (257, 96)])
+def test_noalloc_matches_quantize_act_at_flux_and_ragged_k(M, K):
+    # the FLUX hidden size, and a K that is a multiple of 32 but not of 256
+    # (the last 256-element stage holds padding blocks with zero scales)
+    import precision_gemm_qlinear_b200 as ql
+    w = draw("normal", (256, K), 23, "w", std=0.02)
+    lay = ql.QLinear("nvfp4", "bias", to_dev_bf16(w))
+    x = to_dev_bf16(draw("student_t", (M, K), 33, "x", nu=3, outlier_frac=0.005,
+                         outlier_factor=20.0))
+    ca, sa, cb, sb = _run_both(lay, x, M)
+    kch = ((K + 255) // 256) * 4
+    nsf = ((M + 127) // 128) * kch * 512
+    assert np.array_equal(ca[: M * K // 2].cpu().numpy(), cb[: M * K // 2].cpu().numpy())
+    assert np.array_equal(sa[: nsf + 4].cpu().numpy(), sb[: nsf + 4].cpu().numpy())
+    lay.close()
+
+
+def test_noalloc_at_the_row_maximum():
+    # M == QL_NOALLOC_MAX_ROWS with a small K (32 MB of activations): the
+    # largest accepted call, bit for bit the regular entry point's output
+    import precision_gemm_qlinear_b200 as ql
+    from precision_gemm_qlinear_b200 import _abi
+    M, K = _abi.QL_NOALLOC_MAX_ROWS, 32
+    w = draw("normal", (256, K), 24, "w", std=0.02)
+    lay = ql.QLinear("nvfp4", "bias", to_dev_bf16(w))
+    x = to_dev_bf16(draw("normal", (M, K), 34, "x"))
+    ca, sa, cb, sb = _run_both(lay, x, M)
+    nsf = (M // 128) * 4 * 512
+    assert np.array_equal(ca[: M * K // 2].cpu().numpy(), cb[: M * K // 2].cpu().numpy())
+    assert np.array_equal(sa[: nsf + 4].cpu().numpy(), sb[: nsf + 4].cpu().numpy())
+    lay.close()
+
+
 def test_noalloc_rejects_rows_beyond_the_maximum():
     import precision_gemm_qlinear_b200 as ql
     from precision_gemm_qlinear_b200 import _abi
