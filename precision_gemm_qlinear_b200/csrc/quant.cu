@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
       amb = fmaxf(amb, __shfl_xor_sync(0xffffffffu, amb, 1));  // the block's other half
       const uint32_t sb = cvt_e4m3x2(0.f, __fmul_rn(amb, enc)) & 0xFF;
       const float den = __fmul_rn(e4m3_to_f32(sb), G);
-      const float inv = den > 0.f ? __fdiv_rn(1.f, den) : 0.f;
+      const float inv = den > 0.f ? __frcp_rn(den) : 0.f;  // fl(1/den), correctly rounded
       if (live && vi < nvec)
         qr[vi] = e2m1_4(make_uint2(v[u].x, v[u].y), inv) | (e2m1_4(make_uint2(v[u].z, v[u].w), inv) << 16);
       const uint32_t b1 = __shfl_down_sync(0xffffffffu, sb, 2);
