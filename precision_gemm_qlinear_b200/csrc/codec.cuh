@@ -57,7 +57,7 @@ __device__ __forceinline__ uint32_t nvfp4_block(const uint4& v0, const uint4& v1
   amb = fmaxf(absmax8(v0), absmax8(v1));
   const uint32_t sb = cvt_e4m3x2(0.f, __fmul_rn(amb, enc)) & 0xFF;
   const float den = __fmul_rn(e4m3_to_f32(sb), G);
-  const float inv = den > 0.f ? __frcp_rn(den) : 0.f;  // fl(1/den), correctly rounded
+  const float inv = den > 0.f ? __fdiv_rn(1.f, den) : 0.f;
   codes.x = e2m1_4(make_uint2(v0.x, v0.y), inv) | (e2m1_4(make_uint2(v0.z, v0.w), inv) << 16);
   codes.y = e2m1_4(make_uint2(v1.x, v1.y), inv) | (e2m1_4(make_uint2(v1.z, v1.w), inv) << 16);
   return sb;
