@@ -415,8 +415,11 @@ def _timed_loop(stream, fn, target_ms, min_calls, max_calls=5000):
 def gemm_roofline(model, stream, peaks, peak_src, target_ms):
     """Each layer's GEMM (+ fused epilogue) timed alone over the rotating
     sets (their activation codes were written by the timed steps)."""
+    import torch
     out = []
     nsets = len(model.sets)
+    dev = torch.device(model.dev)
+    dev_index = dev.index if dev.index is not None else 0
     for j, layer in enumerate(model.wl.layers):
         w16 = layer.fmt == "w8a16"
         fused_out = j + 1 < len(model.wl.layers) and model.fused[j + 1]
@@ -426,7 +429,8 @@ def gemm_roofline(model, stream, peaks, peak_src, target_ms):
             codes = model.inputs_of(layers, j) if w16 else layers[j]["codes"]
             model.gemm(j, layers, codes, stream, amax_from=model.sets[(i - 1) % nsets],
                        fused_out=fused_out)
-        ms, n = _timed_loop(stream, run, target_ms, MIN_GEMM_LAUNCHES)
+        with ClockSampler(dev_index, period=0.01) as cs:
+            ms, n = _timed_loop(stream, run, target_ms, MIN_GEMM_LAUNCHES)
         achieved = layer.flops / (ms / 1e3) / 1e12
         sustained = ms * n > 1000.0
         bf16 = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
@@ -439,6 +443,7 @@ def gemm_roofline(model, stream, peaks, peak_src, target_ms):
             "frac": round(achieved / peak, 4), "frac_vs_sustained": round(achieved / peak_sus, 4),
             "traffic": traffic, "traffic_capture": capture,
             "algorithmic_bytes": gemm_bytes(layer), "gemm_ms": round(ms, 5), "launches": n,
+            "clocks": cs.summary(),
             "fused_nvfp4_out": bool(fused_out),
             "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} x "
                            f"{NOMINAL_RATIO[layer.fmt]:g} (nominal {layer.fmt}/bf16 ratio)"})
