@@ -137,58 +137,124 @@ __global__ void __launch_bounds__(256) tensor_amax_kernel(const uint4* __restric
 // are issued before any is used.  Rows are taken in reverse order so that the
 // first ones processed are the tensor's tail, which the amax pass read last
 // and which is still in L2.  Padding rows and K groups get zero scales.
-template <int U>
+//
+// The kernel is issue-bound unless each element costs few instructions, so:
+// the block maximum is taken on bf16 pairs (sign bits cleared, max.bf16x2,
+// which like fmaxf ignores a NaN operand), the element products
+// fl(x * inv_b) are packed f32x2 multiplies (each half rounded as the scalar
+// __fmul_rn), and inv_b = fl(1 / fl(dec(sb) * G)) is looked up in a
+// 128-entry table that every CTA fills once from the tensor factors (sb is a
+// non-negative E4M3 code, 0..0x7F) -- the same values the per-block division
+// gives.  Full steps (all 32 lanes inside the row) run without predicates.
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a & 0x7FFF7FFFu), "r"(b & 0x7FFF7FFFu));
+  return r;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f32x2_splat(float a) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(a));
+  return r;
+}
+// the two values of a bf16x2 word as an f32 pair (element 0 in the low half)
+__device__ __forceinline__ uint64_t bf16x2_f32x2(uint32_t w) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+  return r;
+}
+// 8 bf16 values times inv (per element, rounded) -> 8 E2M1 codes, element 0
+// in the low nibble
+__device__ __forceinline__ uint32_t e2m1_8(const uint4& v, uint64_t inv2) {
+  const uint64_t p0 = mul_f32x2(bf16x2_f32x2(v.x), inv2), p1 = mul_f32x2(bf16x2_f32x2(v.y), inv2);
+  const uint64_t p2 = mul_f32x2(bf16x2_f32x2(v.z), inv2), p3 = mul_f32x2(bf16x2_f32x2(v.w), inv2);
+  uint32_t r;
+  asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t.reg .f32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
+      "mov.b64 {l0, h0}, %1;\n\tmov.b64 {l1, h1}, %2;\n\t"
+      "mov.b64 {l2, h2}, %3;\n\tmov.b64 {l3, h3}, %4;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c0, h0, l0;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c1, h1, l1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c2, h2, l2;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c3, h3, l3;\n\t"
+      "mov.b32 %0, {c0, c1, c2, c3};\n\t}"
+      : "=r"(r)
+      : "l"(p0), "l"(p1), "l"(p2), "l"(p3));
+  return r;
+}
+
+template <int U, int LAYOUT>
 __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
     const __nv_bfloat16* __restrict__ x, int64_t M, int64_t K, int64_t ldx,
-    uint8_t* __restrict__ q, uint8_t* __restrict__ sf, int sf_layout, int64_t bn, int64_t nks,
-    int64_t mpad, const uint32_t* __restrict__ amax_bits, float* g_out, RowMap map) {
+    uint8_t* __restrict__ q, uint8_t* __restrict__ sf, int64_t bn, int64_t nks, int64_t mpad,
+    const uint32_t* __restrict__ amax_bits, float* g_out, RowMap map) {
+  __shared__ float inv_tab[128];
   const int lane = threadIdx.x & 31;
   const int64_t w = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   grid_dep_wait();  // the tensor amax of the previous kernel
   grid_dep_launch_dependents();
-  if (w >= mpad) return;  // warp-uniform
-  const int64_t row = mpad - 1 - w;
   float G, enc;
   nvfp4_tensor_factors(__uint_as_float(*amax_bits), G, enc);
+  if (threadIdx.x < 128) {
+    const float den = __fmul_rn(e4m3_to_f32(threadIdx.x), G);
+    inv_tab[threadIdx.x] = den > 0.f ? __frcp_rn(den) : 0.f;  // fl(1/den), correctly rounded
+  }
+  __syncthreads();
+  if (w >= mpad) return;  // warp-uniform
+  const int64_t row = mpad - 1 - w;
   if (w == 0 && lane == 0 && g_out != nullptr) *g_out = G;
-  const bool live = row < M;
+  // The lane's scale word of step s: activation atoms, 4 groups (2048 bytes)
+  // per step; weights: the replicated chunks (four copies per word).
+  uint32_t* sfa = nullptr;
+  if constexpr (LAYOUT == 0)
+    sfa = reinterpret_cast<uint32_t*>(sf + sf_offset(row, (lane >> 3) * 4, nks * 4));
+  auto put_scale = [&](int64_t s, uint32_t word) {
+    if constexpr (LAYOUT == 0) {
+      sfa[s * 512] = word;
+    } else {
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4)
+        *reinterpret_cast<uint32_t*>(sf + sfb_word_offset(row, s, lane >> 3, q4, nks, bn)) = word;
+    }
+  };
+  if (row >= M) {  // padding row: zero scales
+    if ((lane & 7) == 0)
+      for (int64_t s = 0; s < nks; ++s) put_scale(s, 0u);
+    return;
+  }
   const int64_t nvec = K >> 3;  // 16-byte vectors of a row
-  const uint4* xr = reinterpret_cast<const uint4*>(x + (live ? map(row) : 0) * ldx);
-  uint32_t* qr = reinterpret_cast<uint32_t*>(q + (live ? row : 0) * (K >> 1));
-  for (int64_t s0 = 0; s0 < nks; s0 += U) {
+  const uint4* xr = reinterpret_cast<const uint4*>(x + map(row) * ldx);
+  uint32_t* qr = reinterpret_cast<uint32_t*>(q + row * (K >> 1));
+  // one step: block scale, codes, scale word
+  auto step = [&](int64_t s, const uint4& v, bool code_ok) {
+    const uint32_t m2 = bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w));
+    float amb = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
+    amb = fmaxf(amb, __shfl_xor_sync(0xffffffffu, amb, 1));  // the block's other half
+    const uint32_t sb = cvt_e4m3x2(0.f, __fmul_rn(amb, enc)) & 0x7F;
+    const float inv = inv_tab[sb];
+    const uint64_t inv2 = f32x2_splat(inv);
+    if (code_ok) qr[s * 32 + lane] = e2m1_8(v, inv2);
+    const uint32_t b1 = __shfl_down_sync(0xffffffffu, sb, 2);
+    const uint32_t b2 = __shfl_down_sync(0xffffffffu, sb, 4);
+    const uint32_t b3 = __shfl_down_sync(0xffffffffu, sb, 6);
+    if ((lane & 7) == 0) put_scale(s, sb | (b1 << 8) | (b2 << 16) | (b3 << 24));
+  };
+  const int64_t nfull = nvec >> 5;  // steps with all 32 lanes inside the row
+  int64_t s0 = 0;
+  for (; s0 + U <= nfull; s0 += U) {
     uint4 v[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t vi = (s0 + u) * 32 + lane;
-      v[u] = (live && s0 + u < nks && vi < nvec) ? ld_nc(xr + vi) : make_uint4(0u, 0u, 0u, 0u);
-    }
+    for (int u = 0; u < U; ++u) v[u] = ld_nc(xr + (s0 + u) * 32 + lane);
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (s0 + u >= nks) break;  // warp-uniform
-      const int64_t vi = (s0 + u) * 32 + lane;
-      float amb = absmax8(v[u]);
-      amb = fmaxf(amb, __shfl_xor_sync(0xffffffffu, amb, 1));  // the block's other half
-      const uint32_t sb = cvt_e4m3x2(0.f, __fmul_rn(amb, enc)) & 0xFF;
-      const float den = __fmul_rn(e4m3_to_f32(sb), G);
-      const float inv = den > 0.f ? __frcp_rn(den) : 0.f;  // fl(1/den), correctly rounded
-      if (live && vi < nvec)
-        qr[vi] = e2m1_4(make_uint2(v[u].x, v[u].y), inv) | (e2m1_4(make_uint2(v[u].z, v[u].w), inv) << 16);
-      const uint32_t b1 = __shfl_down_sync(0xffffffffu, sb, 2);
-      const uint32_t b2 = __shfl_down_sync(0xffffffffu, sb, 4);
-      const uint32_t b3 = __shfl_down_sync(0xffffffffu, sb, 6);
-      if ((lane & 7) == 0) {
-        const uint32_t word = sb | (b1 << 8) | (b2 << 16) | (b3 << 24);
-        const int64_t g = (s0 + u) * 4 + (lane >> 3);  // 64-element group of the row
-        if (sf_layout == 0) {
-          *reinterpret_cast<uint32_t*>(sf + sf_offset(row, g * 4, nks * 4)) = word;
-        } else {
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            *reinterpret_cast<uint32_t*>(sf + sfb_word_offset(row, g >> 2, g & 3, q4, nks, bn)) =
-                word;
-        }
-      }
-    }
+    for (int u = 0; u < U; ++u) step(s0 + u, v[u], true);
+  }
+  for (; s0 < nks; ++s0) {  // the rest: partial steps, zero past the row
+    const int64_t vi = s0 * 32 + lane;
+    const bool in = vi < nvec;
+    step(s0, in ? ld_nc(xr + vi) : make_uint4(0u, 0u, 0u, 0u), in);
   }
 }
 
@@ -348,8 +414,12 @@ cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx,
   const int64_t blocks = (mpad + 7) / 8;  // 8 warps (rows) per CTA
   cudaLaunchAttribute at[1];
   cudaLaunchConfig_t c = pdl_config(static_cast<unsigned>(blocks), 256, 0, st, at, 0);
-  return cudaLaunchKernelEx(&c, quant_nvfp4_kernel<4>, static_cast<const __nv_bfloat16*>(x), M, K,
-                            ldx, q, sf, sf_layout, bn, nks, mpad, amax_bits, g_out, map);
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (sf_layout == 0)
+    return cudaLaunchKernelEx(&c, quant_nvfp4_kernel<4, 0>, xb, M, K, ldx, q, sf, bn, nks, mpad,
+                              amax_bits, g_out, map);
+  return cudaLaunchKernelEx(&c, quant_nvfp4_kernel<4, 1>, xb, M, K, ldx, q, sf, bn, nks, mpad,
+                            amax_bits, g_out, map);
 }
 
 cudaError_t launch_debug_encode(int mode, const void* in, int64_t n, const float* amax,
