@@ -1,8 +1,11 @@
-// codec.cuh -- bf16 -> E4M3 / E2M1 encoding steps shared by the quantize
-// kernels and the GEMM epilogue that writes NVFP4 output, so that both produce
-// the same codes from the same bf16 values.  Every float step is an explicitly
-// rounded IEEE operation; the encodes are the hardware's round-to-nearest-even
-// saturating conversions (cvt.rn.satfinite).
+// codec.cuh -- bf16 -> E4M3 / E2M1 encoding steps of the FP8 quantize
+// kernel, of the GEMM epilogue that writes NVFP4 output and of the encoder
+// test hook, and the NVFP4 tensor factors shared with the NVFP4 quantize
+// kernels.  Those compute the same steps on packed pairs (bf16x2 maxima,
+// f32x2 products; each half rounded as the scalar operation), so all produce
+// the same codes from the same bf16 values.  Every float step is an explicitly rounded IEEE
+// operation; the encodes are the hardware's round-to-nearest-even saturating
+// conversions (cvt.rn.satfinite).
 #pragma once
 
 #include <cuda_bf16.h>

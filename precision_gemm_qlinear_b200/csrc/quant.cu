@@ -12,7 +12,10 @@
 //    straight into the GEMM's scale-factor atom layout.
 //
 // Every float step is an explicitly rounded IEEE operation (__fmul_rn /
-// __fdiv_rn) so no FMA contraction changes a code.
+// __fdiv_rn, or mul.rn.f32x2, whose halves round as the scalar multiply) so
+// no FMA contraction changes a code.  The NVFP4 kernels take maxima of |x|
+// on bf16 pairs (max.bf16x2): exact, and like fmaxf they ignore a NaN
+// operand.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -33,6 +36,34 @@ __device__ __forceinline__ uint4 ld_nc(const uint4* p) {
   return v;
 }
 
+// max(|a|, |b|) of two bf16 pairs, pair by pair: sign bits cleared, then
+// max.bf16x2, which (like fmaxf) returns the other operand when one is NaN
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a & 0x7FFF7FFFu), "r"(b & 0x7FFF7FFFu));
+  return r;
+}
+// the two halves of such a pair as one float (the larger)
+__device__ __forceinline__ float bf16x2_hmax(uint32_t m) {
+  return fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xFFFF0000u));
+}
+
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f32x2_splat(float a) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(a));
+  return r;
+}
+// the two values of a bf16x2 word as an f32 pair (element 0 in the low half)
+__device__ __forceinline__ uint64_t bf16x2_f32x2(uint32_t w) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+  return r;
+}
 // ------------------------------------------------------ FP8 per-token quant
 
 // A team of T threads handles one row; 256 / T rows per CTA iteration.  Up to
@@ -99,24 +130,36 @@ __global__ void __launch_bounds__(256, 4) quant_fp8_rows_kernel(const __nv_bfloa
 
 // ------------------------------------------------------------ tensor amax
 
-__global__ void __launch_bounds__(256) tensor_amax_kernel(const uint4* __restrict__ x,
+// Grid-stride |x| maximum over bf16 pairs: U 16-byte loads per thread in
+// flight, a running bf16x2 maximum per load slot (sign bits cleared; NaN
+// operands ignored as fmaxf would), then the pair halves, the warp, the CTA
+// and one atomicMax on the float bits (amax >= 0, so they order as integers).
+template <int U, int CTAS_PER_SM>
+__global__ void __launch_bounds__(256, CTAS_PER_SM) tensor_amax_kernel(const uint4* __restrict__ x,
                                                           int64_t nvec, uint32_t* amax_bits) {
   grid_dep_wait();
   grid_dep_launch_dependents();
-  float m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f;
+  uint32_t m[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) m[u] = 0u;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (; i + 3 * stride < nvec; i += 4 * stride) {
-    uint4 a = ld_nc(x + i), b = ld_nc(x + i + stride), c = ld_nc(x + i + 2 * stride),
-          d = ld_nc(x + i + 3 * stride);
-    m0 = fmaxf(m0, absmax8(a));
-    m1 = fmaxf(m1, absmax8(b));
-    m2 = fmaxf(m2, absmax8(c));
-    m3 = fmaxf(m3, absmax8(d));
+  for (; i + (U - 1) * stride < nvec; i += U * stride) {
+    uint4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) v[u] = ld_nc(x + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      m[u] = bf16x2_absmax(m[u], bf16x2_absmax(bf16x2_absmax(v[u].x, v[u].y),
+                                               bf16x2_absmax(v[u].z, v[u].w)));
   }
-  for (; i < nvec; i += stride) m0 = fmaxf(m0, absmax8(ld_nc(x + i)));
-  const float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-  const uint32_t a = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
+  for (; i < nvec; i += stride) {
+    const uint4 v = ld_nc(x + i);
+    m[0] = bf16x2_absmax(m[0], bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w)));
+  }
+#pragma unroll
+  for (int u = 1; u < U; ++u) m[0] = bf16x2_absmax(m[0], m[u]);
+  const uint32_t a = __reduce_max_sync(0xffffffffu, __float_as_uint(bf16x2_hmax(m[0])));
   __shared__ uint32_t red[8];
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
   __syncthreads();
@@ -146,27 +189,6 @@ __global__ void __launch_bounds__(256) tensor_amax_kernel(const uint4* __restric
 // 128-entry table that every CTA fills once from the tensor factors (sb is a
 // non-negative E4M3 code, 0..0x7F) -- the same values the per-block division
 // gives.  Full steps (all 32 lanes inside the row) run without predicates.
-__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a & 0x7FFF7FFFu), "r"(b & 0x7FFF7FFFu));
-  return r;
-}
-__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ uint64_t f32x2_splat(float a) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(a));
-  return r;
-}
-// the two values of a bf16x2 word as an f32 pair (element 0 in the low half)
-__device__ __forceinline__ uint64_t bf16x2_f32x2(uint32_t w) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
-  return r;
-}
 // 8 bf16 values times inv (per element, rounded) -> 8 E2M1 codes, element 0
 // in the low nibble
 __device__ __forceinline__ uint32_t e2m1_8(const uint4& v, uint64_t inv2) {
@@ -230,8 +252,7 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
   uint32_t* qr = reinterpret_cast<uint32_t*>(q + row * (K >> 1));
   // one step: block scale, codes, scale word
   auto step = [&](int64_t s, const uint4& v, bool code_ok) {
-    const uint32_t m2 = bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w));
-    float amb = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
+    float amb = bf16x2_hmax(bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w)));
     amb = fmaxf(amb, __shfl_xor_sync(0xffffffffu, amb, 1));  // the block's other half
     const uint32_t sb = cvt_e4m3x2(0.f, __fmul_rn(amb, enc)) & 0x7F;
     const float inv = inv_tab[sb];
@@ -396,12 +417,15 @@ cudaError_t launch_tensor_amax(const void* x, int64_t n_elems, uint32_t* amax_bi
                                cudaStream_t st) {
   if (n_elems <= 0) return cudaSuccess;
   const int64_t nvec = n_elems >> 3;
+  // one wave: the grid-stride loop covers the rest
+  constexpr int kU = 8, kCtasPerSm = 6;
   int64_t blocks = (nvec + 255) / 256;
-  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  const int64_t cap = static_cast<int64_t>(num_sms) * kCtasPerSm;
   if (blocks > cap) blocks = cap;
   cudaLaunchAttribute at[1];
   cudaLaunchConfig_t c = pdl_config(static_cast<unsigned>(blocks), 256, 0, st, at, 0);
-  return cudaLaunchKernelEx(&c, tensor_amax_kernel, static_cast<const uint4*>(x), nvec, amax_bits);
+  return cudaLaunchKernelEx(&c, tensor_amax_kernel<kU, kCtasPerSm>, static_cast<const uint4*>(x),
+                            nvec, amax_bits);
 }
 
 cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
