@@ -14,7 +14,8 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libqlinear_b200.so")
 SOURCES = ["quant.cu", "gemm.cu", "noalloc.cu", "qlinear_api.cu"]
-HEADERS = ["ptx.cuh", "internal.h", "codec.cuh", os.path.join("..", "..", "include", "qlinear.h")]
+HEADERS = ["ptx.cuh", "internal.h", "codec.cuh", "amax.cuh",
+           os.path.join("..", "..", "include", "qlinear.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

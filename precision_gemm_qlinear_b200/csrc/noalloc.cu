@@ -18,6 +18,7 @@
 #include <mutex>
 
 #include "../../include/qlinear.h"
+#include "amax.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -54,34 +55,14 @@ uint32_t* scratch_ptr(int dev) {
   return ptrs[dev];
 }
 
-__device__ __forceinline__ float absmax8_bits(const uint4& v) {
-  float m = fmaxf(fabsf(bf16lo(v.x)), fabsf(bf16hi(v.x)));
-  m = fmaxf(m, fmaxf(fabsf(bf16lo(v.y)), fabsf(bf16hi(v.y))));
-  m = fmaxf(m, fmaxf(fabsf(bf16lo(v.z)), fabsf(bf16hi(v.z))));
-  m = fmaxf(m, fmaxf(fabsf(bf16lo(v.w)), fabsf(bf16hi(v.w))));
-  return m;
-}
-
-// Grid-stride max |x| over the whole tensor (M * K / 8 vectors of 8): each
-// CTA writes (does not accumulate) its maximum to partial[blockIdx.x], so no
-// entry has to start at zero.
-__global__ void __launch_bounds__(256) partial_amax_kernel(const uint4* __restrict__ xv,
-                                                           int64_t nvec,
-                                                           uint32_t* __restrict__ partial) {
-  float m = 0.f;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nvec;
-       i += stride)
-    m = fmaxf(m, absmax8_bits(__ldg(xv + i)));
-  uint32_t a = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
-  __shared__ uint32_t red[8];
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    uint32_t b = 0;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) b = max(b, red[w]);
-    partial[blockIdx.x] = b;
-  }
+// Grid-stride max |x| over the whole tensor (M * K / 8 vectors of 8, the
+// same pass as the tensor amax of qlinear_quantize_act): each CTA writes (does
+// not accumulate) its maximum to partial[blockIdx.x], so no entry has to
+// start at zero.
+__global__ void __launch_bounds__(256, kAmaxCtasPerSm) partial_amax_kernel(
+    const uint4* __restrict__ xv, int64_t nvec, uint32_t* __restrict__ partial) {
+  const uint32_t b = cta_max_bits(grid_stride_absmax<kAmaxLoads>(xv, nvec));
+  if (threadIdx.x == 0) partial[blockIdx.x] = b;
 }
 
 // One CTA: tensor amax = max over the nblocks partials, written to *out.
@@ -132,12 +113,12 @@ ql_status quantize_act_noalloc(int fmt, int64_t K, int num_sms, const void* x, i
   if (dev >= kMaxDevices) return QL_ERR_UNSUPPORTED;
   uint32_t* scratch = scratch_ptr(dev);
   if (scratch == nullptr) return QL_ERR_CUDA;
-  // amax pass: up to eight CTAs an SM (never more than the array's partials),
-  // grid-stride over the tensor
+  // amax pass: one wave of up to kAmaxCtasPerSm CTAs an SM (never more than
+  // the array's partials), grid-stride over the tensor
   const int64_t nvec = M * K / 8;
   int64_t nblk = (nvec + 255) / 256;
-  const int64_t cap = static_cast<int64_t>(num_sms) * 8 < kMaxPartials
-                          ? static_cast<int64_t>(num_sms) * 8
+  const int64_t cap = static_cast<int64_t>(num_sms) * kAmaxCtasPerSm < kMaxPartials
+                          ? static_cast<int64_t>(num_sms) * kAmaxCtasPerSm
                           : static_cast<int64_t>(kMaxPartials);
   if (nblk > cap) nblk = cap;
   uint8_t* sf = static_cast<uint8_t*>(scales);

@@ -20,6 +20,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "amax.cuh"
 #include "codec.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -27,26 +28,6 @@
 namespace qlb {
 
 namespace {
-
-__device__ __forceinline__ uint4 ld_nc(const uint4* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-// max(|a|, |b|) of two bf16 pairs, pair by pair: sign bits cleared, then
-// max.bf16x2, which (like fmaxf) returns the other operand when one is NaN
-__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a & 0x7FFF7FFFu), "r"(b & 0x7FFF7FFFu));
-  return r;
-}
-// the two halves of such a pair as one float (the larger)
-__device__ __forceinline__ float bf16x2_hmax(uint32_t m) {
-  return fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xFFFF0000u));
-}
 
 __device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
   uint64_t r;
@@ -96,12 +77,12 @@ __global__ void __launch_bounds__(256, 4) quant_fp8_rows_kernel(const __nv_bfloa
     for (int i = 0; i < VPL; ++i) {
       const int idx = tt + i * T;
       if (valid && idx < nvec) {
-        v[i] = ld_nc(xr + idx);
+        v[i] = ld_nc_v4(xr + idx);
         amax = fmaxf(amax, absmax8(v[i]));
       }
     }
     for (int idx = tt + VPL * T; valid && idx < nvec; idx += T)
-      amax = fmaxf(amax, absmax8(ld_nc(xr + idx)));
+      amax = fmaxf(amax, absmax8(ld_nc_v4(xr + idx)));
     // amax >= 0, so the float bit patterns order like unsigned integers
     uint32_t a = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
     if constexpr (WPT > 1) {
@@ -124,50 +105,23 @@ __global__ void __launch_bounds__(256, 4) quant_fp8_rows_kernel(const __nv_bfloa
       if (valid && idx < nvec) qr[idx] = e4m3_8(v[i], inv);
     }
     for (int idx = tt + VPL * T; valid && idx < nvec; idx += T)
-      qr[idx] = e4m3_8(ld_nc(xr + idx), inv);
+      qr[idx] = e4m3_8(ld_nc_v4(xr + idx), inv);
   }
 }
 
 // ------------------------------------------------------------ tensor amax
 
-// Grid-stride |x| maximum over bf16 pairs: U 16-byte loads per thread in
-// flight, a running bf16x2 maximum per load slot (sign bits cleared; NaN
-// operands ignored as fmaxf would), then the pair halves, the warp, the CTA
-// and one atomicMax on the float bits (amax >= 0, so they order as integers).
+// Grid-stride |x| maximum (grid_stride_absmax: U loads in flight per
+// thread, bf16-pair maxima), then the CTA maximum and one atomicMax on the
+// float bits (amax >= 0, so they order as integers).
 template <int U, int CTAS_PER_SM>
 __global__ void __launch_bounds__(256, CTAS_PER_SM) tensor_amax_kernel(const uint4* __restrict__ x,
-                                                          int64_t nvec, uint32_t* amax_bits) {
+                                                                       int64_t nvec,
+                                                                       uint32_t* amax_bits) {
   grid_dep_wait();
   grid_dep_launch_dependents();
-  uint32_t m[U];
-#pragma unroll
-  for (int u = 0; u < U; ++u) m[u] = 0u;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (; i + (U - 1) * stride < nvec; i += U * stride) {
-    uint4 v[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) v[u] = ld_nc(x + i + u * stride);
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-      m[u] = bf16x2_absmax(m[u], bf16x2_absmax(bf16x2_absmax(v[u].x, v[u].y),
-                                               bf16x2_absmax(v[u].z, v[u].w)));
-  }
-  for (; i < nvec; i += stride) {
-    const uint4 v = ld_nc(x + i);
-    m[0] = bf16x2_absmax(m[0], bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w)));
-  }
-#pragma unroll
-  for (int u = 1; u < U; ++u) m[0] = bf16x2_absmax(m[0], m[u]);
-  const uint32_t a = __reduce_max_sync(0xffffffffu, __float_as_uint(bf16x2_hmax(m[0])));
-  __shared__ uint32_t red[8];
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    uint32_t b = 0;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b = max(b, red[w]);
-    atomicMax(amax_bits, b);
-  }
+  const uint32_t b = cta_max_bits(grid_stride_absmax<U>(x, nvec));
+  if (threadIdx.x == 0) atomicMax(amax_bits, b);
 }
 
 // ------------------------------------------------------- NVFP4 block quant
@@ -252,7 +206,7 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
   uint32_t* qr = reinterpret_cast<uint32_t*>(q + row * (K >> 1));
   // one step: block scale, codes, scale word
   auto step = [&](int64_t s, const uint4& v, bool code_ok) {
-    float amb = bf16x2_hmax(bf16x2_absmax(bf16x2_absmax(v.x, v.y), bf16x2_absmax(v.z, v.w)));
+    float amb = bf16x2_hmax(absmax8_pair(v));
     amb = fmaxf(amb, __shfl_xor_sync(0xffffffffu, amb, 1));  // the block's other half
     const uint32_t sb = cvt_e4m3x2(0.f, __fmul_rn(amb, enc)) & 0x7F;
     const float inv = inv_tab[sb];
@@ -268,14 +222,14 @@ __global__ void __launch_bounds__(256) quant_nvfp4_kernel(
   for (; s0 + U <= nfull; s0 += U) {
     uint4 v[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) v[u] = ld_nc(xr + (s0 + u) * 32 + lane);
+    for (int u = 0; u < U; ++u) v[u] = ld_nc_v4(xr + (s0 + u) * 32 + lane);
 #pragma unroll
     for (int u = 0; u < U; ++u) step(s0 + u, v[u], true);
   }
   for (; s0 < nks; ++s0) {  // the rest: partial steps, zero past the row
     const int64_t vi = s0 * 32 + lane;
     const bool in = vi < nvec;
-    step(s0, in ? ld_nc(xr + vi) : make_uint4(0u, 0u, 0u, 0u), in);
+    step(s0, in ? ld_nc_v4(xr + vi) : make_uint4(0u, 0u, 0u, 0u), in);
   }
 }
 
@@ -418,14 +372,13 @@ cudaError_t launch_tensor_amax(const void* x, int64_t n_elems, uint32_t* amax_bi
   if (n_elems <= 0) return cudaSuccess;
   const int64_t nvec = n_elems >> 3;
   // one wave: the grid-stride loop covers the rest
-  constexpr int kU = 8, kCtasPerSm = 6;
   int64_t blocks = (nvec + 255) / 256;
-  const int64_t cap = static_cast<int64_t>(num_sms) * kCtasPerSm;
+  const int64_t cap = static_cast<int64_t>(num_sms) * kAmaxCtasPerSm;
   if (blocks > cap) blocks = cap;
   cudaLaunchAttribute at[1];
   cudaLaunchConfig_t c = pdl_config(static_cast<unsigned>(blocks), 256, 0, st, at, 0);
-  return cudaLaunchKernelEx(&c, tensor_amax_kernel<kU, kCtasPerSm>, static_cast<const uint4*>(x),
-                            nvec, amax_bits);
+  return cudaLaunchKernelEx(&c, tensor_amax_kernel<kAmaxLoads, kAmaxCtasPerSm>,
+                            static_cast<const uint4*>(x), nvec, amax_bits);
 }
 
 cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
