@@ -392,10 +392,21 @@ cudaError_t launch_quant_nvfp4(const void* x, int64_t M, int64_t K, int64_t ldx,
   cudaLaunchAttribute at[1];
   cudaLaunchConfig_t c = pdl_config(static_cast<unsigned>(blocks), 256, 0, st, at, 0);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  if (sf_layout == 0)
-    return cudaLaunchKernelEx(&c, quant_nvfp4_kernel<4, 0>, xb, M, K, ldx, q, sf, bn, nks, mpad,
+  if (sf_layout == 1)  // weights, once per layer
+    return cudaLaunchKernelEx(&c, quant_nvfp4_kernel<4, 1>, xb, M, K, ldx, q, sf, bn, nks, mpad,
                               amax_bits, g_out, map);
-  return cudaLaunchKernelEx(&c, quant_nvfp4_kernel<4, 1>, xb, M, K, ldx, q, sf, bn, nks, mpad,
+  // Activations: as many loads in flight as divide the row's 256-element
+  // steps evenly (a remainder runs one step at a time), 8 (76 registers,
+  // 3 CTAs an SM) or 6 (64 registers, 4 CTAs) before 4: e.g. K = 3072
+  // (12 steps) takes 6, K = 8192 and 12288 take 8.
+  const int64_t nfull = K >> 8;  // steps with all 32 lanes inside the row
+  if (nfull >= 8 && nfull % 8 == 0)
+    return cudaLaunchKernelEx(&c, quant_nvfp4_kernel<8, 0>, xb, M, K, ldx, q, sf, bn, nks, mpad,
+                              amax_bits, g_out, map);
+  if (nfull >= 6 && nfull % 6 == 0)
+    return cudaLaunchKernelEx(&c, quant_nvfp4_kernel<6, 0>, xb, M, K, ldx, q, sf, bn, nks, mpad,
+                              amax_bits, g_out, map);
+  return cudaLaunchKernelEx(&c, quant_nvfp4_kernel<4, 0>, xb, M, K, ldx, q, sf, bn, nks, mpad,
                             amax_bits, g_out, map);
 }
 
