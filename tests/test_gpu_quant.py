@@ -37,8 +37,14 @@ def test_fp8_act_quant_bitexact(M, K):
     assert np.array_equal(gc, rc)
 
 
+# The block pass keeps 8, 6 or 4 steps of 256 elements in flight (the most
+# that divide the row's full steps) and runs a remainder one step at a time;
+# the shapes cover each depth with and without a remainder: 32 / 256 / 544
+# (4, remainder only), 3072 (6), 3168 (6 + a partial step), 12288 (8),
+# 8224 (8 + a partial step).
 @pytest.mark.parametrize("M,K,dist", [(1, 32, "n"), (128, 256, "t"), (300, 3072, "t"),
-                                      (257, 544, "n"), (64, 12288, "t")])
+                                      (257, 544, "n"), (64, 12288, "t"), (129, 3168, "t"),
+                                      (40, 8224, "n")])
 def test_nvfp4_act_quant_bitexact(M, K, dist):
     import torch
     lay, _ = _layer("nvfp4", 256, K)
