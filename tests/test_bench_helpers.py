@@ -76,3 +76,35 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert _bench(["--impl", "reference", "--steps", "1", "--warmup", "0",
                    "--workload", "tiny_fp8"],
                   {"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_recorded_traffic_matches_the_algorithmic_bytes_it_was_scaled_by():
+    # profiles/traffic.json records, beside each capture, the algorithmic
+    # bytes of the captured launch and of the benchmark's launch; they must
+    # be the bench's own figures, and a capture of a smaller M is scaled by
+    # exactly their ratio (the weight re-reads grow with M)
+    import dataclasses
+    import json
+    import os
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)
+    for key, e in rec.items():
+        name, _, j = key.partition(":")
+        layer = WORKLOADS[name].layers[int(j)]
+        assert e["kernel"].startswith("qgemm_kernel<" + layer.fmt + ",")
+        assert os.path.exists(os.path.join(bench.ROOT, e["capture"]))
+        b, cap = bench.profiled_traffic(name, int(j), layer.M)
+        fresh = e["source_sha"] == bench.gemm_source_sha()
+        assert (b is not None) == fresh
+        if "M" in e:
+            small = dataclasses.replace(layer, M=e["M"])
+            assert e["algorithmic_bytes_captured"] == bench.gemm_bytes(small)
+            assert e["algorithmic_bytes_full"] == bench.gemm_bytes(layer)
+            if fresh:
+                ratio = e["algorithmic_bytes_full"] / e["algorithmic_bytes_captured"]
+                assert b == int(float(e["dram_bytes_per_launch"]) * ratio)
+                assert cap == e["capture"]
+        else:
+            assert e["algorithmic_bytes"] == bench.gemm_bytes(layer)
+            if fresh:
+                assert b == e["dram_bytes_per_launch"]
