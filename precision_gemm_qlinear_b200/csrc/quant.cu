@@ -11,9 +11,9 @@
 //    scale per 16 K-elements, packed E2M1 codes; block scales are written
 //    straight into the GEMM's scale-factor atom layout.
 //
-// Every float step is an explicitly rounded IEEE operation (__fmul_rn /
-// __fdiv_rn, or mul.rn.f32x2, whose halves round as the scalar multiply) so
-// no FMA contraction changes a code.  The NVFP4 kernels take maxima of |x|
+// Every float step is an explicitly rounded IEEE operation (__fmul_rn,
+// __fdiv_rn, __frcp_rn, or mul.rn.f32x2, whose halves round as the scalar
+// multiply) so no FMA contraction changes a code.  The NVFP4 kernels take maxima of |x|
 // on bf16 pairs (max.bf16x2): exact, and like fmaxf they ignore a NaN
 // operand.
 #include <cuda_bf16.h>
@@ -29,22 +29,6 @@ namespace qlb {
 
 namespace {
 
-__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ uint64_t f32x2_splat(float a) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(a));
-  return r;
-}
-// the two values of a bf16x2 word as an f32 pair (element 0 in the low half)
-__device__ __forceinline__ uint64_t bf16x2_f32x2(uint32_t w) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
-  return r;
-}
 // ------------------------------------------------------ FP8 per-token quant
 
 // A team of T threads handles one row; 256 / T rows per CTA iteration.  Up to
@@ -143,6 +127,24 @@ __global__ void __launch_bounds__(256, CTAS_PER_SM) tensor_amax_kernel(const uin
 // 128-entry table that every CTA fills once from the tensor factors (sb is a
 // non-negative E4M3 code, 0..0x7F) -- the same values the per-block division
 // gives.  Full steps (all 32 lanes inside the row) run without predicates.
+// packed f32x2 helpers: one instruction per pair, each half rounded as the
+// scalar operation
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f32x2_splat(float a) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(a));
+  return r;
+}
+// the two values of a bf16x2 word as an f32 pair (element 0 in the low half)
+__device__ __forceinline__ uint64_t bf16x2_f32x2(uint32_t w) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+  return r;
+}
 // 8 bf16 values times inv (per element, rounded) -> 8 E2M1 codes, element 0
 // in the low nibble
 __device__ __forceinline__ uint32_t e2m1_8(const uint4& v, uint64_t inv2) {
